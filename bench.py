@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon optimizer step (GPT-2 124M: 48 hidden matrices) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gpt2_124m]
+
+One JSON line on stdout (rank 0).  A "step" is one full Muon optimizer step
+over all matrices of the workload: momentum + Nesterov + Frobenius norm + bf16
+cast (one kernel), 5 quintic Newton-Schulz iterations (Gram, polynomial and
+X-update kernels, grouped over all matrices), and the fused parameter update.
+
+* value     ms per step, inputs resident in HBM, CUDA events on the launching
+            stream around exactly K steps (barrier + synchronize on both
+            sides, max over ranks).  Gradients cycle through 4 pre-generated
+            sets (1.36 GB, larger than L2), so no step reads a warm L2.
+* e2e       the same step through the public API from pinned host memory:
+            every step copies its gradients host->device and reads the
+            updated parameters back device->host inside the timed region.
+* roofline  the dominant kernel (largest share of device time), timed live
+            with CUDA events bracketing each of its launches in the timed
+            region, against MEASURED_PEAKS.json.
+* cpu_baseline  the CPU oracle (fp64 NumPy, emulated bf16) on a bounded sample
+            (one GPT-2 block, 4 matrices), scaled to the full step.
+
+Under torchrun (N > 1) every rank runs its own independent 48-matrix step on
+its own GPU with its own seed (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, WorkloadStream  # noqa: E402
+
+METRIC = "Muon step ms, GPT-2 124M 48 mats; Newton-Schulz bf16 TFLOP/s vs tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+N_GRAD_SETS = 4
+KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="gpt2_124m", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(wl):
+    shapes = sorted(set(wl.shapes), key=lambda s: wl.shapes.index(s))
+    return {
+        "workload": f"{wl.name}: {wl.n_matrices} fp32 matrices "
+                    f"({', '.join(f'{r}x{c}' for r, c in shapes)}), "
+                    f"grads rank-{wl.grad_rank} + {wl.grad_noise} noise, "
+                    f"momentum N(0,{wl.buf_std}^2), lr {wl.lr}, beta {wl.beta}, "
+                    f"nesterov, {wl.ns_steps} NS steps, coeffs {list(wl.coeffs)}",
+        "matrices": wl.n_matrices,
+        "elements": wl.n_elements,
+        "ns_flop_per_step": wl.ns_flops(),
+        "l2": f"inputs larger than L2: {N_GRAD_SETS} gradient sets cycled "
+              f"({N_GRAD_SETS * wl.n_elements * 4 / 1e9:.2f} GB) + params + momentum",
+        "precision": "fp32 momentum/norm/update; Newton-Schulz bf16 operands, fp32 accumulation",
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"],
+                    source="fallback")
+
+
+# ---------------------------------------------------------------- algorithmic work per launch
+
+def per_launch_work(wl):
+    """Algorithmic FLOPs (tensor kernels) or bytes (HBM kernels) per launch."""
+    g = p = u = 0.0
+    for r, c in wl.shapes:
+        m, n = min(r, c), max(r, c)
+        g += m * m * n          # Gram, upper triangle
+        p += m ** 3             # symmetric square
+        u += 2 * m * m * n      # X update
+    el = wl.n_elements
+    return {
+        "momentum_norm_cast": ("hbm", 14.0 * el),     # read g, buf; write buf (fp32); write X0 (bf16)
+        "gram": ("tensor", g),
+        "poly": ("tensor", p),
+        "xupdate": ("tensor", u),
+        "xupdate_final": ("tensor", u),
+        "apply": ("hbm", 10.0 * el),
+    }
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "newton_schulz_norm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != source_hash():
+        return None
+    ent = d.get("kernels", {}).get(kind)
+    return None if ent is None else float(ent["bytes_per_launch"])
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_oracle_block(wl, params, grads, bufs, idx):
+    """Time the oracle on the given matrices (one step); returns seconds."""
+    from oracle import muon_step_ref
+    t0 = time.perf_counter()
+    muon_step_ref([params[i] for i in idx], [grads[i] for i in idx], [bufs[i] for i in idx],
+                  lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps,
+                  coeffs=wl.coeffs)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, wl, rank):
+    """Reference arm: the CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return 0
+    st = WorkloadStream(wl, seed=0, subset=[0, 1, 2, 3])
+    params, bufs = st.init()
+    grads = st.next_grads()
+    per_shape = {0: [], 1: [], 2: [], 3: []}
+    steps = max(args.steps, 4)
+    for k in range(args.warmup + steps):
+        i = k % 4
+        t = cpu_oracle_block(wl, params, grads, bufs, [i])
+        if k >= args.warmup:
+            per_shape[i].append(t)
+    block_s = sum(statistics.mean(v) for v in per_shape.values())
+    ms = 1e3 * block_s * (wl.n_matrices / 4)
+    cores = blas_threads()
+    out = {
+        "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl),
+        "cpu_baseline": {"value": ms, "unit": "ms", "cores": cores, "kind": "oracle",
+                         "sample": "each step runs the oracle on one matrix of the first GPT-2 "
+                                   "block (cycling its 4 shapes); ms/step = 12 x the summed "
+                                   "per-shape mean"},
+        "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def flat_views(torch, shapes, device, dtype, pinned=False):
+    """One contiguous buffer with a 64-element-aligned view per matrix."""
+    offs, tot = [], 0
+    for r, c in shapes:
+        offs.append(tot)
+        tot += (r * c + 63) // 64 * 64
+    if device == "cpu":
+        flat = torch.empty(tot, dtype=dtype, pin_memory=pinned)
+    else:
+        flat = torch.empty(tot, dtype=dtype, device=device)
+    views = [flat[o:o + r * c].view(r, c) for o, (r, c) in zip(offs, shapes)]
+    return flat, views
+
+
+def run_ours(args, wl, rank, world):
+    import torch
+    import newton_schulz_norm_b200 as muon
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- inputs (seeded per rank), resident in HBM
+    st = WorkloadStream(wl, seed=rank)
+    params, bufs = st.init()
+    grad_sets = [st.next_grads() for _ in range(N_GRAD_SETS)]
+
+    # CPU oracle baseline on a bounded sample (rank 0, N = 1 only), before GPU work
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        idx = [0, 1, 2, 3]
+        secs = cpu_oracle_block(wl, params, grad_sets[0], bufs, idx)
+        cpu_base = {"value": 1e3 * secs * wl.n_matrices / len(idx), "unit": "ms",
+                    "cores": blas_threads(), "kind": "oracle",
+                    "sample": f"oracle on matrices {idx} (one GPT-2 block), 1 step, "
+                              f"{secs:.1f} s, scaled x{wl.n_matrices // len(idx)} to the full step"}
+
+    shapes = list(wl.shapes)
+    p_flat, P = flat_views(torch, shapes, dev, torch.float32)
+    b_flat, B = flat_views(torch, shapes, dev, torch.float32)
+    g_flats, G = [], []
+    for gs in grad_sets:
+        f, v = flat_views(torch, shapes, dev, torch.float32)
+        for t, a in zip(v, gs):
+            t.copy_(torch.from_numpy(a))
+        g_flats.append(f)
+        G.append(v)
+    for t, a in zip(P, params):
+        t.copy_(torch.from_numpy(a))
+    for t, a in zip(B, bufs):
+        t.copy_(torch.from_numpy(a))
+    torch.cuda.synchronize()
+
+    kw = dict(lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    stream = torch.cuda.current_stream()
+
+    for w in range(args.warmup):
+        muon.step(P, G[w % N_GRAD_SETS], B, **kw)
+    torch.cuda.synchronize()
+    if muon.status() != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    # ---- timed region (device-resident)
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    muon.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        muon.step(P, G[k % N_GRAD_SETS], B, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = muon.profile_end()
+    barrier()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local)
+    if muon.status() != 0:
+        raise RuntimeError("device-side error in the timed region")
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    hg = []
+    for gs in grad_sets:
+        f, v = flat_views(torch, shapes, "cpu", torch.float32, pinned=True)
+        for t, a in zip(v, gs):
+            t.copy_(torch.from_numpy(a))
+        hg.append(f)
+    hp, _ = flat_views(torch, shapes, "cpu", torch.float32, pinned=True)
+    torch.cuda.synchronize()
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for k in range(e2e_steps):
+        g_flats[0].copy_(hg[k % N_GRAD_SETS], non_blocking=True)
+        muon.step(P, G[0], B, **kw)
+        hp.copy_(p_flat, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3) / e2e_steps)
+
+    # ---- roofline of the dominant kernel
+    peaks = load_peaks()
+    work = per_launch_work(wl)
+    dom = max((k for k in KINDS if prof[k][1] > 0), key=lambda k: prof[k][0])
+    bound, per_launch = work[dom]
+    avg_ms = prof[dom][0] / prof[dom][1]
+    if bound == "tensor":
+        achieved = per_launch / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = per_launch / (avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": recorded_traffic(dom),
+                "peak_source": f"{peaks['source']} (burst)",
+                "work_per_launch": per_launch, "avg_launch_ms": avg_ms}
+
+    kernels = {}
+    for k in KINDS:
+        tot, n = prof[k]
+        if n == 0:
+            continue
+        b, wpl = work[k]
+        rate = wpl / (tot / n * 1e-3)
+        kernels[k] = {"launches": n, "ms_per_launch": tot / n, "share": None,
+                      ("tflops" if b == "tensor" else "gbs"): rate / (1e12 if b == "tensor" else 1e9)}
+    tot_all = sum(prof[k][0] for k in KINDS)
+    for k in kernels:
+        kernels[k]["share"] = prof[k][0] / tot_all
+    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "xupdate", "xupdate_final")) / args.steps
+    ns_tflops = wl.ns_flops() / (ns_ms * 1e-3) / 1e12
+    launches = sum(prof[k][1] for k in KINDS)
+
+    out = {
+        "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "ns_tflops": ns_tflops, "ns_frac_of_peak": ns_tflops / peaks["bf16_tflops"],
+        "ns_ms_per_step": ns_ms,
+        "roofline": roofline, "kernels": kernels,
+        "cpu_baseline": cpu_base,
+        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * wl.n_elements,
+                "d2h_bytes_per_step": 4 * wl.n_elements, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl, rank)
+    return run_ours(args, wl, rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * muon.h -- C interface of the B200 (sm_100a) Muon optimizer step.
+ *
+ * The Muon step (X thread "New training speed record for @karpathy's
+ * 124M-parameter NanoGPT setup", tweets 2/8, 5/8 and 6/8) orthogonalises, for
+ * every 2-D parameter, the SGD-Nesterov momentum update with a quintic
+ * Newton-Schulz iteration run in bfloat16.  Per matrix of stored shape r x c:
+ *
+ *   buf <- beta*buf + g                       momentum, PyTorch convention
+ *                                             ("07. Training neural networks",
+ *                                             section "Momentum")
+ *   u    = g + beta*buf   (nesterov != 0)     Nesterov look-ahead (tweet 5/8)
+ *   u    = buf            (nesterov == 0)
+ *   X0   = bf16(u / (||u||_F + 1e-7))         Frobenius normalisation
+ *   X0  <- X0^T if r > c                      orient so that rows <= cols
+ *   repeat ns_steps times (tweets 5/8, 6/8):
+ *     A  = bf16(X X^T)                        fp32 accumulation
+ *     B  = bf16(b*A + c*A*A)
+ *     X  = bf16(a*X + B*X)
+ *   X   <- X^T if r > c
+ *   p   <- p - (lr*sqrt(max(1, r/c))) * X     one fp32 rounding per element
+ *
+ * Default coefficients (a, b, c) = (3.4445, -4.7750, 2.0315).
+ *
+ * Conventions for every entry point:
+ *  - Matrices are fp32 (or bf16 where stated), row-major, contiguous
+ *    (leading dimension = number of columns), on the current CUDA device.
+ *  - "pointer arrays" are HOST arrays whose entries are DEVICE pointers.
+ *  - Device pointers must be 16-byte aligned (else MUON_ERR_UNSUPPORTED).
+ *  - stream is a cudaStream_t passed as void*; NULL means the legacy default
+ *    stream.  Calls are asynchronous: they return after enqueueing; results
+ *    are valid in stream order.  At most one call in flight per stream.
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and leave every buffer untouched.  n = 0 is a no-op returning MUON_OK.
+ *  - Device-side failures (a bounded wait that ran out) never hang: the
+ *    kernel records MUON_ERR_TIMEOUT in a per-device status word, which
+ *    muon_status() reports.
+ *  - NaN/Inf in one matrix's gradient propagate to that matrix only.
+ *  - The library owns its scratch memory (bf16 iterates, Gram matrices,
+ *    norm partials), cached per device and shape set, allocated with
+ *    cudaMalloc on the first call for a shape set and freed by
+ *    muon_release().  The caller owns params, grads, bufs and streams.
+ *  - Thread safety: the plan cache is guarded by a mutex; distinct streams
+ *    may be used from distinct host threads, but two calls sharing one shape
+ *    set share scratch memory and must be ordered on the GPU (same stream).
+ */
+#ifndef MUON_H_
+#define MUON_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = -1,  /* null pointer, bad size, non-finite scalar   */
+  MUON_ERR_UNSUPPORTED = -2,  /* misaligned pointer, no sm_100 device, ...   */
+  MUON_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed            */
+  MUON_ERR_NOMEM = -4,        /* cudaMalloc of scratch memory failed          */
+  MUON_ERR_TIMEOUT = -5       /* a device-side bounded wait ran out           */
+} muon_status_t;
+
+/* Largest number of matrices one muon_step call groups into a single
+ * launch sequence; larger n is processed in consecutive groups. */
+#define MUON_MAX_GROUP 512
+
+/*
+ * muon_step -- one Muon optimizer step over n 2-D parameters.
+ *
+ *   params  pointer array [n]: fp32 r_i x c_i, updated in place.
+ *   grads   pointer array [n]: fp32 r_i x c_i, read only.
+ *   bufs    pointer array [n]: fp32 r_i x c_i momentum buffers, updated in
+ *           place (the optimizer's only state).
+ *   shapes  host int64 array [2n]: r_0, c_0, r_1, c_1, ...; all > 0 and
+ *           r*c < 2^31.
+ *   lr      learning rate (finite); beta momentum (finite).
+ *   nesterov  non-zero: u = g + beta*buf; zero: u = buf.
+ *   ns_steps  Newton-Schulz iterations, 0..100 (0: X = X0).
+ *   coeffs  host float[3] (a, b, c), or NULL for the default triple.
+ *   stream  cudaStream_t as void*.
+ * params, grads and bufs must not alias one another or across matrices.
+ * Returns MUON_OK or a negative muon_status_t.
+ */
+MUON_API int muon_step(float* const* params, const float* const* grads, float* const* bufs,
+              const int64_t* shapes, int n, float lr, float beta, int nesterov,
+              int ns_steps, const float* coeffs, void* stream);
+
+/*
+ * muon_orthogonalize -- the Newton-Schulz part alone, for one matrix:
+ *   out = NS(bf16(x / (||x||_F + 1e-7)))   (orientation handled as above)
+ *
+ *   x      device fp32 rows x cols (read only).
+ *   out    device rows x cols, fp32 (out_is_bf16 == 0) or bf16 bits
+ *          (out_is_bf16 != 0); may not alias x.
+ * Same coefficient, step and stream rules as muon_step.
+ */
+MUON_API int muon_orthogonalize(const float* x, void* out, int out_is_bf16, int64_t rows,
+                       int64_t cols, int ns_steps, const float* coeffs, void* stream);
+
+/*
+ * Stage entry points: each runs one kernel of the step on caller buffers, so
+ * that every stage can be checked on its own.  bf16 buffers hold raw bf16
+ * bits (uint16_t), row-major with leading dimension ld (elements, ld >= the
+ * row length, ld % 8 == 0).
+ */
+
+/* muon_momentum_normalize -- the fused first kernel for n matrices:
+ *   buf <- beta*buf + g;  u = g + beta*buf (or buf);
+ *   x0  = bf16(u / (||u||_F + 1e-7)), written ORIENTED (min(r,c) rows,
+ *         max(r,c) columns, leading dimension x0_ld[i]) to x0[i].
+ * x0 is a pointer array of device bf16 buffers; x0_ld a host int64 array. */
+MUON_API int muon_momentum_normalize(const float* const* grads, float* const* bufs,
+                            uint16_t* const* x0, const int64_t* x0_ld,
+                            const int64_t* shapes, int n, float beta, int nesterov,
+                            void* stream);
+
+/* muon_gram -- a = bf16(x x^T); x: m x n (ld_x), a: m x m (ld_a). */
+MUON_API int muon_gram(const uint16_t* x, int64_t ld_x, uint16_t* a, int64_t ld_a,
+              int64_t m, int64_t n, void* stream);
+
+/* muon_poly -- b_out = bf16(cb*a + cc*(a a)); a: symmetric m x m. */
+MUON_API int muon_poly(const uint16_t* a, int64_t ld_a, uint16_t* b_out, int64_t ld_b,
+              int64_t m, float cb, float cc, void* stream);
+
+/* muon_xupdate -- x_out = bf16(ca*x + b x); b: m x m, x, x_out: m x n.
+ * x_out may not alias x. */
+MUON_API int muon_xupdate(const uint16_t* b, int64_t ld_b, const uint16_t* x, int64_t ld_x,
+                 uint16_t* x_out, int64_t ld_out, int64_t m, int64_t n, float ca,
+                 void* stream);
+
+/* muon_status -- synchronises the stream, then returns (and clears) the
+ * device-side status of the current device: MUON_OK or MUON_ERR_TIMEOUT;
+ * MUON_ERR_CUDA if the synchronisation itself failed. */
+MUON_API int muon_status(void* stream);
+
+/* muon_error_string -- static description of a status code. */
+MUON_API const char* muon_error_string(int code);
+
+/* muon_set_wait_limit_ns -- bound for every device-side wait (default
+ * 2e9 ns; read from MUON_SPIN_LIMIT_NS at load time if set).  0 makes every
+ * wait that does not succeed at once give up, for fault tests. */
+MUON_API void muon_set_wait_limit_ns(uint64_t ns);
+
+/* muon_workspace_bytes -- scratch bytes muon_step would allocate for this
+ * shape set (host-only computation; no allocation). */
+MUON_API int64_t muon_workspace_bytes(const int64_t* shapes, int n);
+
+/*
+ * Per-kernel timing, for measurement.  Between muon_profile_begin() and
+ * muon_profile_end() every kernel this library launches is bracketed by a
+ * pair of CUDA events recorded on its own stream (cudaEventRecord is
+ * asynchronous; the kernels themselves are unchanged).  muon_profile_end()
+ * synchronises those events and writes, per kernel kind, the summed device
+ * time in milliseconds and the launch count:
+ *   0 momentum/norm/cast   1 Gram   2 polynomial   3 X update
+ *   4 X update with the fused parameter update   5 update without NS steps
+ * ms and launches are host arrays of at least nkinds entries.  Returns the
+ * number of kinds written, or a negative status.
+ */
+#define MUON_PROFILE_KINDS 6
+MUON_API void muon_profile_begin(void);
+MUON_API int muon_profile_end(double* ms, int64_t* launches, int nkinds);
+
+/* muon_release -- synchronises the device and frees every cached plan and
+ * scratch buffer of every device this process used. */
+MUON_API void muon_release(void);
+
+/* muon_version -- library version string. */
+MUON_API const char* muon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_H_ */

@@ -1,0 +1,144 @@
+// internal.h -- data structures shared by the host planner and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "muon.h"
+
+namespace muon {
+
+// ---------------------------------------------------------------- NS GEMM tiling
+// One CTA computes a BM x BN output tile with tcgen05.mma M=128, N=256, K=16,
+// fed by TMA through a STAGES-deep ring of BK-wide K slices.
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                      // one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int BOX = 64;                     // TMA box: 64 x 64 bf16 = 8 KB
+constexpr int BOX_BYTES = BOX * BOX * 2;
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int GEMM_THREADS = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int EPI_THREADS = 128;
+constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators of BN columns
+constexpr int GEMM_BAR_BYTES = 256;
+constexpr size_t GEMM_SMEM_BYTES = size_t(STAGES) * STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
+
+enum NsOp : int { OP_GRAM = 0, OP_POLY = 1, OP_UPDATE = 2 };
+
+// What the X-update epilogue does with X_{k+1}.
+enum FinalMode : int {
+  FINAL_NONE = 0,      // store bf16 X_{k+1} to the next iterate buffer
+  FINAL_PARAM = 1,     // p <- p - scale * X_{k+1}   (fp32, stored orientation)
+  FINAL_OUT_F32 = 2,   // out <- X_{k+1} as fp32     (stored orientation)
+  FINAL_OUT_BF16 = 3,  // out <- X_{k+1} as bf16     (stored orientation)
+};
+
+// One matrix of one GEMM phase.  Lives in device memory; 64-byte aligned
+// because the tensor maps inside are read by TMA from global memory.
+struct alignas(64) NsProblem {
+  CUtensorMap tmA;            // A operand source: K-major rows x K
+  CUtensorMap tmB;            // B operand source: K-major (Gram, poly) or MN-major (update)
+  const __nv_bfloat16* epi;   // poly: A (for b*A); update: X (for a*X)
+  __nv_bfloat16* out;         // bf16 output (A, B or X_{k+1})
+  long long ld_epi;
+  long long ld_out;
+  int M, N, K;                // output M x N, reduction length K
+  int transposed;             // final modes: output (i, j) lands at [j][i]
+  long long ld_final;         // leading dimension of the final target
+  int slot;                   // index into FinalTable
+  int pad_[3];
+};
+
+struct NsTile {
+  int prob;   // index into the NsProblem array
+  int i0;     // first output row
+  int j0;     // first output column
+  int kc;     // number of BK slices
+};
+
+struct FinalTable {
+  void* ptr[MUON_MAX_GROUP];
+  float scale[MUON_MAX_GROUP];
+};
+
+struct NsLaunch {
+  const NsProblem* probs;
+  const NsTile* tiles;
+  int ntiles;
+  int final_mode;
+  float ca, cb, cc;
+  unsigned long long limit_ns;
+  int* status;
+};
+
+// ---------------------------------------------------------------- fused first kernel
+// Momentum + Nesterov + Frobenius norm + bf16 cast + orientation, over
+// 64 x 64 tiles of the stored matrix, in two passes joined per matrix.
+constexpr int K1_TILE = 64;
+constexpr int K1_THREADS = 256;
+
+enum K1Mode : int { K1_MOMENTUM = 0, K1_PLAIN = 1 };
+
+struct K1Info {              // static per matrix (device memory)
+  long long r, c;            // stored shape
+  long long ldx;             // leading dimension of the oriented bf16 X0
+  int tiles_c;               // tiles along the stored columns
+  int ntiles;                // tiles of this matrix
+  int part0;                 // offset of its partial sums
+  int transposed;            // r > c
+};
+
+struct K1Ptrs {              // per call
+  const float* g;            // gradient (or the matrix to orthogonalise)
+  float* buf;                // momentum buffer (unused in K1_PLAIN)
+  __nv_bfloat16* x0;         // oriented bf16 output
+};
+
+// Work item: pass in bit 31, matrix in bits [16,31), tile in [0,16) would be
+// too small for big matrices, so items are two ints.
+struct K1Item {
+  int mat;                   // matrix index; pass 2 items have mat | 0x40000000
+  int tile;
+};
+constexpr int K1_PASS2 = 0x40000000;
+
+struct K1Launch {
+  const K1Info* info;
+  const K1Item* items;
+  int nitems;
+  int mode;
+  int nesterov;
+  float beta;
+  int* counter;              // work-queue head (zeroed before launch)
+  int* done;                 // [n] pass-1 tiles finished (zeroed)
+  int* ready;                // [n] norm published (zeroed)
+  double* partials;          // per tile sum of squares
+  double* norms;             // [n] Frobenius norms
+  unsigned long long limit_ns;
+  int* status;
+  K1Ptrs ptrs[MUON_MAX_GROUP];
+};
+
+// Applies p <- p - scale * X0 when ns_steps == 0 (no GEMM epilogue to fuse into).
+struct ApplyLaunch {
+  const K1Info* info;
+  int n;
+  int mode;                  // FINAL_PARAM / FINAL_OUT_F32 / FINAL_OUT_BF16
+  K1Ptrs ptrs[MUON_MAX_GROUP];   // x0 = source, g unused
+  void* dst[MUON_MAX_GROUP];
+  float scale[MUON_MAX_GROUP];
+};
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
+                           cudaStream_t stream);
+cudaError_t ns_gemm_setup(int device);
+cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);
+cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream);
+
+}  // namespace muon

@@ -1,0 +1,266 @@
+// momentum.cu -- the HBM-bound first kernel of the Muon step, and the
+// elementwise update used when no Newton-Schulz iteration runs.
+//
+// Per matrix (stored r x c, fp32):
+//   buf <- beta*buf + g                 ("07. Training neural networks",
+//                                        section "Momentum": PyTorch form)
+//   u    = g + beta*buf  (Nesterov)     (X thread, tweet 5/8: orthogonalise
+//   u    = buf           (plain)         the update after Nesterov momentum)
+//   nu   = ||u||_F
+//   X0   = bf16(u / (nu + 1e-7)), stored transposed when r > c.
+//
+// The norm needs the whole matrix before any element can be cast, so the
+// kernel works in two passes over 64 x 64 tiles, fed by one work queue:
+//   pass 1 (tile): momentum, write buf, partial sum of squares;
+//   pass 2 (tile): wait until the matrix's norm is published, recompute u
+//                  from g and the new buf, scale, cast, (transpose,) store.
+// The queue holds pass 1 of matrix i+1 between passes 1 and 2 of matrix i, so
+// pass 2 normally re-reads g and buf from L2, and only the one matrix whose
+// norm is pending waits.  The last pass-1 tile of a matrix sums the partials
+// in a fixed order (deterministic norm) and publishes it with a release
+// store.  Pass-2 tiles are queued after every pass-1 tile of their matrix, so
+// a waiting CTA only ever waits on CTAs that are already running; the wait is
+// still bounded and reports MUON_ERR_TIMEOUT instead of hanging.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace muon {
+
+namespace {
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();  // red may still be read by the previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double t = 0.0;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < K1_THREADS / 32; ++w) t += red[w];   // fixed order
+  }
+  return t;  // valid in thread 0 only
+}
+
+__device__ __forceinline__ float momentum_u(float g, float& b, float beta, int mode, int nesterov) {
+  if (mode == K1_PLAIN) return g;
+  b = fmaf(beta, b, g);
+  return nesterov ? fmaf(beta, b, g) : b;
+}
+
+__device__ __forceinline__ float u_from(float g, float bnew, float beta, int mode, int nesterov) {
+  if (mode == K1_PLAIN) return g;
+  return nesterov ? fmaf(beta, bnew, g) : bnew;
+}
+
+__global__ void __launch_bounds__(K1_THREADS) k1_kernel(const __grid_constant__ K1Launch L) {
+  __shared__ int s_item;
+  __shared__ int s_flag;
+  __shared__ double s_norm;
+  __shared__ double s_red[K1_THREADS / 32];
+  __shared__ uint16_t s_tile[K1_TILE][K1_TILE + 2];
+
+  const int tid = threadIdx.x;
+  const int lrow = tid >> 4;         // 0..15
+  const int lcol = (tid & 15) * 4;   // 0..60
+
+  for (;;) {
+    if (tid == 0) s_item = atomicAdd(L.counter, 1);
+    __syncthreads();
+    const int it = s_item;
+    __syncthreads();
+    if (it >= L.nitems) break;
+    const K1Item item = L.items[it];
+    const bool pass2 = (item.mat & K1_PASS2) != 0;
+    const int mat = item.mat & ~K1_PASS2;
+    const K1Info info = L.info[mat];
+    const K1Ptrs P = L.ptrs[mat];
+    const long long r = info.r, c = info.c;
+    const long long r0 = (long long)(item.tile / info.tiles_c) * K1_TILE;
+    const long long c0 = (long long)(item.tile % info.tiles_c) * K1_TILE;
+    const bool vec = (c & 3) == 0;
+    const float beta = L.beta;
+
+    if (!pass2) {
+      double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const long long gr = r0 + lrow + 16 * k;
+        const long long gc = c0 + lcol;
+        if (gr >= r || gc >= c) continue;
+        const long long off = gr * c + gc;
+        if (vec && gc + 4 <= c) {
+          const float4 g4 = __ldg(reinterpret_cast<const float4*>(P.g + off));
+          float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+          float bv[4] = {0.f, 0.f, 0.f, 0.f};
+          float4 b4;
+          if (L.mode != K1_PLAIN) {
+            b4 = *reinterpret_cast<const float4*>(P.buf + off);
+            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+          }
+          float s = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float u = momentum_u(gv[e], bv[e], beta, L.mode, L.nesterov);
+            s = fmaf(u, u, s);
+          }
+          ss += (double)s;
+          if (L.mode != K1_PLAIN)
+            *reinterpret_cast<float4*>(P.buf + off) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+        } else {
+          for (int e = 0; e < 4 && gc + e < c; ++e) {
+            float b = (L.mode != K1_PLAIN) ? P.buf[off + e] : 0.f;
+            const float u = momentum_u(P.g[off + e], b, beta, L.mode, L.nesterov);
+            ss += (double)u * (double)u;
+            if (L.mode != K1_PLAIN) P.buf[off + e] = b;
+          }
+        }
+      }
+      const double tot = block_sum(ss, s_red);
+      if (tid == 0) {
+        L.partials[info.part0 + item.tile] = tot;
+        __threadfence();
+        const int prev = atomicAdd(L.done + mat, 1);
+        s_flag = (prev == info.ntiles - 1);
+      }
+      __syncthreads();
+      if (s_flag) {
+        // Last tile of this matrix: fixed-order sum of its partials.
+        __threadfence();
+        double acc = 0.0;
+        for (int t = tid; t < info.ntiles; t += K1_THREADS) acc += __ldcg(L.partials + info.part0 + t);
+        const double all = block_sum(acc, s_red);
+        if (tid == 0) {
+          L.norms[mat] = sqrt(all);
+          __threadfence();
+          st_release_gpu(L.ready + mat, 1);
+        }
+      }
+      continue;
+    }
+
+    // ---------------------------------------------------------------- pass 2
+    if (tid == 0) {
+      int ok = ld_acquire_gpu(L.ready + mat);
+      if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        while (!(ok = ld_acquire_gpu(L.ready + mat))) {
+          if (global_timer_ns() - t0 > L.limit_ns) break;
+          __nanosleep(128);
+        }
+      }
+      if (!ok) atomicCAS(L.status, 0, MUON_ERR_TIMEOUT);
+      s_flag = ok;
+      s_norm = ok ? __ldcg(L.norms + mat) : 0.0;
+    }
+    __syncthreads();
+    if (!s_flag) continue;
+    const double inv = 1.0 / (s_norm + 1e-7);
+    const bool tr = info.transposed != 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int row = lrow + 16 * k;
+      const long long gr = r0 + row;
+      const long long gc = c0 + lcol;
+      uint16_t bits[4] = {0, 0, 0, 0};
+      if (gr < r && gc < c) {
+        const long long off = gr * c + gc;
+        if (vec && gc + 4 <= c) {
+          const float4 g4 = __ldg(reinterpret_cast<const float4*>(P.g + off));
+          float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (L.mode != K1_PLAIN) b4 = __ldcg(reinterpret_cast<const float4*>(P.buf + off));
+          const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float u = u_from(gv[e], bv[e], beta, L.mode, L.nesterov);
+            bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
+          }
+        } else {
+          for (int e = 0; e < 4 && gc + e < c; ++e) {
+            const float b = (L.mode != K1_PLAIN) ? __ldcg(P.buf + off + e) : 0.f;
+            const float u = u_from(P.g[off + e], b, beta, L.mode, L.nesterov);
+            bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
+          }
+        }
+        if (!tr) {
+          __nv_bfloat16* dst = P.x0 + gr * info.ldx + gc;
+          if (gc + 4 <= c) {
+            uint2 w;
+            w.x = (uint32_t)bits[0] | ((uint32_t)bits[1] << 16);
+            w.y = (uint32_t)bits[2] | ((uint32_t)bits[3] << 16);
+            *reinterpret_cast<uint2*>(dst) = w;
+          } else {
+            for (int e = 0; e < 4 && gc + e < c; ++e) dst[e] = __ushort_as_bfloat16(bits[e]);
+          }
+        }
+      }
+      if (tr) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_tile[row][lcol + e] = bits[e];
+      }
+    }
+    if (tr) {
+      __syncthreads();
+      // X0 row (c0 + oc) holds stored column c0 + oc; 8 threads per row.
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int oc = (tid >> 3) + 32 * k2;
+        const int seg = (tid & 7) * 8;
+        const long long xr = c0 + oc;     // row of X0 (= stored column)
+        const long long xc = r0 + seg;    // first column of X0 (= stored row)
+        if (xr >= c || xc >= r) continue;
+        __nv_bfloat16* dst = P.x0 + xr * info.ldx + xc;
+        if (xc + 8 <= r) {
+          uint4 w;
+          w.x = (uint32_t)s_tile[seg + 0][oc] | ((uint32_t)s_tile[seg + 1][oc] << 16);
+          w.y = (uint32_t)s_tile[seg + 2][oc] | ((uint32_t)s_tile[seg + 3][oc] << 16);
+          w.z = (uint32_t)s_tile[seg + 4][oc] | ((uint32_t)s_tile[seg + 5][oc] << 16);
+          w.w = (uint32_t)s_tile[seg + 6][oc] | ((uint32_t)s_tile[seg + 7][oc] << 16);
+          *reinterpret_cast<uint4*>(dst) = w;
+        } else {
+          for (int e = 0; e < 8 && xc + e < r; ++e) dst[e] = __ushort_as_bfloat16(s_tile[seg + e][oc]);
+        }
+      }
+    }
+  }
+}
+
+// p <- p - scale * X0 (or a plain copy of X0 out) for ns_steps == 0.
+__global__ void apply_kernel(const __grid_constant__ ApplyLaunch L) {
+  const int mat = blockIdx.y;
+  if (mat >= L.n) return;
+  const K1Info info = L.info[mat];
+  const long long r = info.r, c = info.c, total = r * c;
+  const __nv_bfloat16* x0 = L.ptrs[mat].x0;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long i = e / c, j = e % c;                 // stored position
+    const long long xo = info.transposed ? (j * info.ldx + i) : (i * info.ldx + j);
+    const float x = __bfloat162float(x0[xo]);
+    if (L.mode == FINAL_PARAM) {
+      float* p = reinterpret_cast<float*>(L.dst[mat]) + e;
+      *p = fmaf(-L.scale[mat], x, *p);
+    } else if (L.mode == FINAL_OUT_F32) {
+      reinterpret_cast<float*>(L.dst[mat])[e] = x;
+    } else {
+      reinterpret_cast<__nv_bfloat16*>(L.dst[mat])[e] = __float2bfloat16_rn(x);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream) {
+  if (L.nitems <= 0) return cudaSuccess;
+  k1_kernel<<<grid, K1_THREADS, 0, stream>>>(L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream) {
+  if (L.n <= 0) return cudaSuccess;
+  apply_kernel<<<dim3(256, L.n), 256, 0, stream>>>(L);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

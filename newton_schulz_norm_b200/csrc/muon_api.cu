@@ -1,0 +1,928 @@
+// muon_api.cu -- the C interface declared in include/muon.h.
+//
+// Host side only: argument checks, the per-device plan cache (scratch
+// buffers, TMA tensor maps, tile lists, work queues) and the launch sequence
+//
+//   K1 (momentum + norm + cast)  ->  [GRAM -> POLY -> UPDATE] x ns_steps
+//
+// where the last UPDATE applies the parameter update in its epilogue.  All
+// matrices of a call share each launch (grouped by phase), so the many small
+// GPT-2 matrices fill the GPU together.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace muon {
+namespace {
+
+constexpr float kDefaultCoeffs[3] = {3.4445f, -4.7750f, 2.0315f};
+constexpr int kMaxSteps = 100;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mutex;
+unsigned long long g_limit_ns = 2000000000ull;
+bool g_limit_from_env = false;
+
+long long round_up(long long v, long long m) { return (v + m - 1) / m * m; }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: rows x cols, row pitch ld elements, 64x64 boxes,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BOX, (cuuint32_t)BOX};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- device memory arena
+
+struct Arena {
+  size_t off = 0;
+  size_t take(size_t bytes, size_t align = 256) {
+    off = (off + align - 1) / align * align;
+    size_t at = off;
+    off += bytes;
+    return at;
+  }
+};
+
+struct DevBlock {
+  char* ptr = nullptr;
+  size_t bytes = 0;
+  ~DevBlock() {
+    if (ptr) cudaFree(ptr);
+  }
+};
+
+// ---------------------------------------------------------------- plans
+
+struct Geom {
+  long long r, c, m, n, ldx, lda;
+  int transposed;
+};
+
+struct NsPhase {
+  NsProblem* probs = nullptr;  // device
+  NsTile* tiles = nullptr;     // device
+  int ntiles = 0;
+};
+
+struct K1Plan {
+  K1Info* info = nullptr;
+  K1Item* items = nullptr;
+  int nitems = 0;
+  int* counters = nullptr;  // [1 + 2n]: head, done[n], ready[n]
+  double* partials = nullptr;
+  double* norms = nullptr;
+  int n = 0;
+};
+
+struct Plan {
+  std::vector<Geom> geom;
+  DevBlock mem;
+  __nv_bfloat16* X[2] = {nullptr, nullptr};  // ping-pong iterates (base of all matrices)
+  std::vector<long long> x_off, a_off;       // per-matrix offsets (elements)
+  __nv_bfloat16* A = nullptr;
+  __nv_bfloat16* B = nullptr;
+  NsPhase gram[2], poly, upd[2];
+  K1Plan k1;
+};
+
+struct DeviceCtx {
+  int device = -1;
+  int num_sms = 0;
+  int k1_blocks_per_sm = 1;
+  int* status = nullptr;
+  std::map<std::vector<long long>, std::unique_ptr<Plan>> plans;
+  std::map<std::vector<long long>, std::unique_ptr<Plan>> stage_plans;
+};
+
+std::map<int, std::unique_ptr<DeviceCtx>> g_ctx;
+
+// ---------------------------------------------------------------- profiling events
+enum ProfKind : int { PK_K1 = 0, PK_GRAM = 1, PK_POLY = 2, PK_UPDATE = 3, PK_FINAL = 4, PK_APPLY = 5 };
+
+struct ProfRecord {
+  int kind;
+  cudaEvent_t start, stop;
+};
+
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+
+Profiler g_prof;
+
+// Records an event pair around one launch when profiling is on.
+struct ProfScope {
+  int kind;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr;
+  ProfScope(int k, cudaStream_t s) : kind(k), stream(s) {
+    if (g_prof.on) {
+      start = g_prof.get();
+      if (start) cudaEventRecord(start, stream);
+    }
+  }
+  ~ProfScope() {
+    if (!start) return;
+    cudaEvent_t stop = g_prof.get();
+    if (!stop) return;
+    cudaEventRecord(stop, stream);
+    g_prof.recs.push_back({kind, start, stop});
+  }
+};
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA; }
+
+int get_ctx(DeviceCtx** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+  auto it = g_ctx.find(dev);
+  if (it != g_ctx.end()) {
+    *out = it->second.get();
+    return MUON_OK;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prop.major != 10) return MUON_ERR_UNSUPPORTED;   // built for sm_100a only
+  if (!encode_fn()) return MUON_ERR_UNSUPPORTED;
+  std::unique_ptr<DeviceCtx> ctx(new DeviceCtx());
+  ctx->device = dev;
+  ctx->num_sms = prop.multiProcessorCount;
+  if (cudaMalloc(&ctx->status, sizeof(int)) != cudaSuccess) return MUON_ERR_NOMEM;
+  if (cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return MUON_ERR_CUDA;
+  if (ns_gemm_setup(dev) != cudaSuccess) return MUON_ERR_CUDA;
+  ctx->k1_blocks_per_sm = 4;
+  *out = ctx.get();
+  g_ctx[dev] = std::move(ctx);
+  return MUON_OK;
+}
+
+unsigned long long limit_ns() {
+  if (!g_limit_from_env) {
+    g_limit_from_env = true;
+    const char* s = std::getenv("MUON_SPIN_LIMIT_NS");
+    if (s && *s) g_limit_ns = std::strtoull(s, nullptr, 10);
+  }
+  return g_limit_ns;
+}
+
+// Gram / poly tiles: only tiles holding some entry on or above the diagonal.
+void sym_tiles(std::vector<NsTile>& t, int prob, long long m, int kc) {
+  for (long long i0 = 0; i0 < m; i0 += BM)
+    for (long long j0 = 0; j0 < m; j0 += BN)
+      if (std::min(j0 + BN - 1, m - 1) >= i0) t.push_back({prob, (int)i0, (int)j0, kc});
+}
+
+void full_tiles(std::vector<NsTile>& t, int prob, long long m, long long n, int kc) {
+  for (long long i0 = 0; i0 < m; i0 += BM)
+    for (long long j0 = 0; j0 < n; j0 += BN) t.push_back({prob, (int)i0, (int)j0, kc});
+}
+
+// K1 work queue: pass 1 of matrix i+1 sits between passes 1 and 2 of matrix i.
+void k1_items(std::vector<K1Item>& items, const std::vector<K1Info>& info) {
+  const int n = (int)info.size();
+  auto p1 = [&](int i) {
+    for (int t = 0; t < info[i].ntiles; ++t) items.push_back({i, t});
+  };
+  auto p2 = [&](int i) {
+    for (int t = 0; t < info[i].ntiles; ++t) items.push_back({i | K1_PASS2, t});
+  };
+  if (n == 0) return;
+  p1(0);
+  for (int i = 1; i < n; ++i) {
+    p1(i);
+    p2(i - 1);
+  }
+  p2(n - 1);
+}
+
+std::vector<K1Info> k1_infos(const std::vector<Geom>& geom, const std::vector<long long>& ldx) {
+  std::vector<K1Info> info;
+  int part = 0;
+  for (size_t i = 0; i < geom.size(); ++i) {
+    K1Info k;
+    k.r = geom[i].r;
+    k.c = geom[i].c;
+    k.ldx = ldx[i];
+    k.tiles_c = (int)cdiv(k.c, K1_TILE);
+    k.ntiles = (int)(cdiv(k.r, K1_TILE) * k.tiles_c);
+    k.part0 = part;
+    k.transposed = geom[i].transposed;
+    part += k.ntiles;
+    info.push_back(k);
+  }
+  return info;
+}
+
+// Tile lists of the three GEMM phases for a shape set.
+struct TileLists {
+  std::vector<NsTile> gram, poly, upd;
+};
+
+TileLists plan_tiles(const std::vector<Geom>& geom) {
+  TileLists t;
+  const int n = (int)geom.size();
+  for (int i = 0; i < n; ++i) sym_tiles(t.gram, i, geom[i].m, (int)cdiv(geom[i].n, BK));
+  // Longest reduction first so the static round-robin ends evenly.
+  std::stable_sort(t.gram.begin(), t.gram.end(),
+                   [](const NsTile& x, const NsTile& y) { return x.kc > y.kc; });
+  for (int i = 0; i < n; ++i) sym_tiles(t.poly, i, geom[i].m, (int)cdiv(geom[i].m, BK));
+  for (int i = 0; i < n; ++i) full_tiles(t.upd, i, geom[i].m, geom[i].n, (int)cdiv(geom[i].m, BK));
+  return t;
+}
+
+// Byte offsets of every scratch region inside the plan's one allocation.
+struct Layout {
+  long long xel = 0, ael = 0;   // elements of all iterates / all m x m matrices
+  size_t x0 = 0, x1 = 0, a = 0, b = 0, probs = 0, gt = 0, pt = 0, ut = 0;
+  size_t k1info = 0, k1items = 0, counters = 0, partials = 0, norms = 0;
+  size_t k1tiles = 0;
+  size_t total = 0;
+};
+
+Layout plan_layout(const std::vector<Geom>& geom, bool with_ns, const TileLists* t) {
+  Layout L;
+  Arena a;
+  const int n = (int)geom.size();
+  for (const Geom& g : geom) {
+    L.xel += round_up(g.m * g.ldx, 128);
+    L.ael += round_up(g.m * g.lda, 128);
+    L.k1tiles += cdiv(g.r, K1_TILE) * cdiv(g.c, K1_TILE);
+  }
+  L.x0 = a.take(L.xel * 2);
+  if (with_ns) {
+    L.x1 = a.take(L.xel * 2);
+    L.a = a.take(L.ael * 2);
+    L.b = a.take(L.ael * 2);
+    L.probs = a.take(sizeof(NsProblem) * n * 5, 128);
+    L.gt = a.take(sizeof(NsTile) * t->gram.size());
+    L.pt = a.take(sizeof(NsTile) * t->poly.size());
+    L.ut = a.take(sizeof(NsTile) * t->upd.size());
+  }
+  L.k1info = a.take(sizeof(K1Info) * n);
+  L.k1items = a.take(sizeof(K1Item) * 2 * L.k1tiles);
+  L.counters = a.take(sizeof(int) * (1 + 2 * n));
+  L.partials = a.take(sizeof(double) * L.k1tiles);
+  L.norms = a.take(sizeof(double) * n);
+  L.total = a.off;
+  return L;
+}
+
+size_t plan_bytes(const std::vector<Geom>& geom, bool with_ns) {
+  TileLists t;
+  if (with_ns) t = plan_tiles(geom);
+  return plan_layout(geom, with_ns, &t).total;
+}
+
+std::vector<Geom> make_geom(const int64_t* shapes, int n) {
+  std::vector<Geom> geom(n);
+  for (int i = 0; i < n; ++i) {
+    Geom& g = geom[i];
+    g.r = shapes[2 * i];
+    g.c = shapes[2 * i + 1];
+    g.transposed = g.r > g.c;
+    g.m = std::min(g.r, g.c);
+    g.n = std::max(g.r, g.c);
+    g.ldx = round_up(g.n, 8);
+    g.lda = round_up(g.m, 8);
+  }
+  return geom;
+}
+
+int upload_phase(NsPhase& ph, char* base, size_t prob_off, size_t tile_off,
+                 const std::vector<NsProblem>& probs, const std::vector<NsTile>& tiles) {
+  ph.probs = reinterpret_cast<NsProblem*>(base + prob_off);
+  ph.tiles = reinterpret_cast<NsTile*>(base + tile_off);
+  ph.ntiles = (int)tiles.size();
+  if (cudaMemcpy(ph.probs, probs.data(), sizeof(NsProblem) * probs.size(), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (!tiles.empty() &&
+      cudaMemcpy(ph.tiles, tiles.data(), sizeof(NsTile) * tiles.size(), cudaMemcpyHostToDevice) !=
+          cudaSuccess)
+    return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+// Builds the scratch memory, tensor maps, tile lists and work queue for a
+// shape set.  with_ns=false builds only the first-kernel part.
+int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan>* out) {
+  std::unique_ptr<Plan> P(new Plan());
+  P->geom = geom;
+  const int n = (int)geom.size();
+  TileLists tl;
+  if (with_ns) tl = plan_tiles(geom);
+  const Layout lay = plan_layout(geom, with_ns, &tl);
+  if (cudaMalloc(&P->mem.ptr, lay.total) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_NOMEM;
+  }
+  P->mem.bytes = lay.total;
+  char* base = P->mem.ptr;
+  long long xel = 0, ael = 0;
+  P->x_off.resize(n);
+  P->a_off.resize(n);
+  for (int i = 0; i < n; ++i) {
+    P->x_off[i] = xel;
+    P->a_off[i] = ael;
+    xel += round_up(geom[i].m * geom[i].ldx, 128);
+    ael += round_up(geom[i].m * geom[i].lda, 128);
+  }
+  P->X[0] = reinterpret_cast<__nv_bfloat16*>(base + lay.x0);
+  if (with_ns) {
+    P->X[1] = reinterpret_cast<__nv_bfloat16*>(base + lay.x1);
+    P->A = reinterpret_cast<__nv_bfloat16*>(base + lay.a);
+    P->B = reinterpret_cast<__nv_bfloat16*>(base + lay.b);
+    const size_t prob_off = lay.probs;
+    const std::vector<NsTile>& gt = tl.gram;
+    const std::vector<NsTile>& pt = tl.poly;
+    const std::vector<NsTile>& ut = tl.upd;
+    const size_t gt_off = lay.gt, pt_off = lay.pt, ut_off = lay.ut;
+
+    std::vector<NsProblem> pr(n);
+    for (int par = 0; par < 2; ++par) {
+      // Gram: A = X X^T from X[par]
+      for (int i = 0; i < n; ++i) {
+        const Geom& g = geom[i];
+        NsProblem& q = pr[i];
+        std::memset(&q, 0, sizeof(q));
+        const __nv_bfloat16* x = P->X[par] + P->x_off[i];
+        if (!make_map(&q.tmA, x, g.m, g.n, g.ldx)) return MUON_ERR_CUDA;
+        q.tmB = q.tmA;
+        q.out = P->A + P->a_off[i];
+        q.ld_out = g.lda;
+        q.M = (int)g.m;
+        q.N = (int)g.m;
+        q.K = (int)g.n;
+        q.slot = i;
+      }
+      int rc = upload_phase(P->gram[par], base, prob_off + sizeof(NsProblem) * n * par, gt_off, pr, gt);
+      if (rc) return rc;
+      // Update: X[1-par] = a X[par] + B X[par]
+      for (int i = 0; i < n; ++i) {
+        const Geom& g = geom[i];
+        NsProblem& q = pr[i];
+        std::memset(&q, 0, sizeof(q));
+        const __nv_bfloat16* x = P->X[par] + P->x_off[i];
+        if (!make_map(&q.tmA, P->B + P->a_off[i], g.m, g.m, g.lda)) return MUON_ERR_CUDA;
+        if (!make_map(&q.tmB, x, g.m, g.n, g.ldx)) return MUON_ERR_CUDA;
+        q.epi = x;
+        q.ld_epi = g.ldx;
+        q.out = P->X[1 - par] + P->x_off[i];
+        q.ld_out = g.ldx;
+        q.M = (int)g.m;
+        q.N = (int)g.n;
+        q.K = (int)g.m;
+        q.transposed = g.transposed;
+        q.ld_final = g.c;
+        q.slot = i;
+      }
+      rc = upload_phase(P->upd[par], base, prob_off + sizeof(NsProblem) * n * (2 + par), ut_off, pr, ut);
+      if (rc) return rc;
+    }
+    // Poly: B = b A + c A A^T
+    for (int i = 0; i < n; ++i) {
+      const Geom& g = geom[i];
+      NsProblem& q = pr[i];
+      std::memset(&q, 0, sizeof(q));
+      const __nv_bfloat16* am = P->A + P->a_off[i];
+      if (!make_map(&q.tmA, am, g.m, g.m, g.lda)) return MUON_ERR_CUDA;
+      q.tmB = q.tmA;
+      q.epi = am;
+      q.ld_epi = g.lda;
+      q.out = P->B + P->a_off[i];
+      q.ld_out = g.lda;
+      q.M = (int)g.m;
+      q.N = (int)g.m;
+      q.K = (int)g.m;
+      q.slot = i;
+    }
+    int rc = upload_phase(P->poly, base, prob_off + sizeof(NsProblem) * n * 4, pt_off, pr, pt);
+    if (rc) return rc;
+  }
+  // First kernel.
+  std::vector<long long> ldx(n);
+  for (int i = 0; i < n; ++i) ldx[i] = geom[i].ldx;
+  std::vector<K1Info> info = k1_infos(geom, ldx);
+  std::vector<K1Item> items;
+  k1_items(items, info);
+  P->k1.n = n;
+  P->k1.info = reinterpret_cast<K1Info*>(base + lay.k1info);
+  P->k1.items = reinterpret_cast<K1Item*>(base + lay.k1items);
+  P->k1.nitems = (int)items.size();
+  P->k1.counters = reinterpret_cast<int*>(base + lay.counters);
+  P->k1.partials = reinterpret_cast<double*>(base + lay.partials);
+  P->k1.norms = reinterpret_cast<double*>(base + lay.norms);
+  if (cudaMemcpy(P->k1.info, info.data(), sizeof(K1Info) * n, cudaMemcpyHostToDevice) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (cudaMemcpy(P->k1.items, items.data(), sizeof(K1Item) * items.size(), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  *out = std::move(P);
+  return MUON_OK;
+}
+
+int check_shapes(const int64_t* shapes, int n) {
+  if (n < 0 || n > (1 << 20)) return MUON_ERR_INVALID_ARG;
+  if (n > 0 && !shapes) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const long long r = shapes[2 * i], c = shapes[2 * i + 1];
+    if (r <= 0 || c <= 0) return MUON_ERR_INVALID_ARG;
+    if (r * c >= (1ll << 31) || r >= (1ll << 30) || c >= (1ll << 30)) return MUON_ERR_UNSUPPORTED;
+  }
+  return MUON_OK;
+}
+
+int check_coeffs(const float* coeffs, float* co) {
+  const float* src = coeffs ? coeffs : kDefaultCoeffs;
+  for (int i = 0; i < 3; ++i) {
+    if (!std::isfinite(src[i])) return MUON_ERR_INVALID_ARG;
+    co[i] = src[i];
+  }
+  return MUON_OK;
+}
+
+int get_plan(DeviceCtx* ctx, std::vector<long long> key, const std::vector<Geom>& geom, bool with_ns,
+             Plan** out) {
+  auto it = ctx->plans.find(key);
+  if (it != ctx->plans.end()) {
+    *out = it->second.get();
+    return MUON_OK;
+  }
+  std::unique_ptr<Plan> P;
+  int rc = build_plan(geom, with_ns, &P);
+  if (rc) return rc;
+  *out = P.get();
+  ctx->plans[key] = std::move(P);
+  return MUON_OK;
+}
+
+int k1_grid(DeviceCtx* ctx, int nitems) {
+  return std::max(1, std::min(nitems, ctx->num_sms * ctx->k1_blocks_per_sm));
+}
+
+int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, int nesterov,
+           cudaStream_t stream) {
+  const int n = P->k1.n;
+  if (cudaMemsetAsync(P->k1.counters, 0, sizeof(int) * (1 + 2 * n), stream) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  static thread_local K1Launch L;   // large (12 KB); kept off the stack
+  L.info = P->k1.info;
+  L.items = P->k1.items;
+  L.nitems = P->k1.nitems;
+  L.mode = mode;
+  L.nesterov = nesterov;
+  L.beta = beta;
+  L.counter = P->k1.counters;
+  L.done = P->k1.counters + 1;
+  L.ready = P->k1.counters + 1 + n;
+  L.partials = P->k1.partials;
+  L.norms = P->k1.norms;
+  L.limit_ns = limit_ns();
+  L.status = ctx->status;
+  for (int i = 0; i < n; ++i) L.ptrs[i] = ptrs[i];
+  ProfScope ps(PK_K1, stream);
+  return cuda_err(launch_k1(L, k1_grid(ctx, L.nitems), stream));
+}
+
+// The Newton-Schulz chain; the last update writes `final_mode` through F.
+int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mode,
+           const FinalTable* F, cudaStream_t stream) {
+  NsLaunch L;
+  L.ca = co[0];
+  L.cb = co[1];
+  L.cc = co[2];
+  L.limit_ns = limit_ns();
+  L.status = ctx->status;
+  for (int s = 0; s < ns_steps; ++s) {
+    const int par = s & 1;
+    L.final_mode = FINAL_NONE;
+    L.probs = P->gram[par].probs;
+    L.tiles = P->gram[par].tiles;
+    L.ntiles = P->gram[par].ntiles;
+    cudaError_t e;
+    {
+      ProfScope ps(PK_GRAM, stream);
+      e = launch_ns_gemm(OP_GRAM, L, nullptr, std::min(L.ntiles, ctx->num_sms), stream);
+    }
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    L.probs = P->poly.probs;
+    L.tiles = P->poly.tiles;
+    L.ntiles = P->poly.ntiles;
+    {
+      ProfScope ps(PK_POLY, stream);
+      e = launch_ns_gemm(OP_POLY, L, nullptr, std::min(L.ntiles, ctx->num_sms), stream);
+    }
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    L.probs = P->upd[par].probs;
+    L.tiles = P->upd[par].tiles;
+    L.ntiles = P->upd[par].ntiles;
+    L.final_mode = (s == ns_steps - 1) ? final_mode : FINAL_NONE;
+    {
+      ProfScope ps(L.final_mode == FINAL_NONE ? PK_UPDATE : PK_FINAL, stream);
+      e = launch_ns_gemm(OP_UPDATE, L, F, std::min(L.ntiles, ctx->num_sms), stream);
+    }
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+  }
+  return MUON_OK;
+}
+
+int run_apply(Plan* P, int mode, void* const* dst, const float* scale, cudaStream_t stream) {
+  static thread_local ApplyLaunch A;
+  A.info = P->k1.info;
+  A.n = P->k1.n;
+  A.mode = mode;
+  for (int i = 0; i < A.n; ++i) {
+    A.ptrs[i].g = nullptr;
+    A.ptrs[i].buf = nullptr;
+    A.ptrs[i].x0 = P->X[0] + P->x_off[i];
+    A.dst[i] = dst[i];
+    A.scale[i] = scale ? scale[i] : 0.f;
+  }
+  ProfScope ps(PK_APPLY, stream);
+  return cuda_err(launch_apply(A, stream));
+}
+
+std::vector<long long> shape_key(char kind, const std::vector<Geom>& geom) {
+  std::vector<long long> key;
+  key.push_back(kind);
+  for (const Geom& g : geom) {
+    key.push_back(g.r);
+    key.push_back(g.c);
+  }
+  return key;
+}
+
+int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, float* const* bufs,
+               const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
+               const float* co, cudaStream_t stream) {
+  std::vector<Geom> geom = make_geom(shapes, n);
+  Plan* P = nullptr;
+  int rc = get_plan(ctx, shape_key('S', geom), geom, true, &P);
+  if (rc) return rc;
+  std::vector<K1Ptrs> ptrs(n);
+  static thread_local FinalTable F;
+  for (int i = 0; i < n; ++i) {
+    ptrs[i].g = grads[i];
+    ptrs[i].buf = bufs[i];
+    ptrs[i].x0 = P->X[0] + P->x_off[i];
+    F.ptr[i] = params[i];
+    const double s = std::sqrt(std::max(1.0, (double)geom[i].r / (double)geom[i].c));
+    F.scale[i] = (float)((double)lr * s);
+  }
+  rc = run_k1(ctx, P, ptrs.data(), K1_MOMENTUM, beta, nesterov, stream);
+  if (rc) return rc;
+  if (ns_steps == 0) {
+    std::vector<void*> dst(params, params + n);
+    return run_apply(P, FINAL_PARAM, dst.data(), F.scale, stream);
+  }
+  return run_ns(ctx, P, ns_steps, co, FINAL_PARAM, &F, stream);
+}
+
+}  // namespace
+}  // namespace muon
+
+using namespace muon;
+
+extern "C" {
+
+int muon_step(float* const* params, const float* const* grads, float* const* bufs,
+              const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
+              const float* coeffs, void* stream) {
+  int rc = check_shapes(shapes, n);
+  if (rc) return rc;
+  if (n == 0) return MUON_OK;
+  if (!params || !grads || !bufs) return MUON_ERR_INVALID_ARG;
+  if (!std::isfinite(lr) || !std::isfinite(beta)) return MUON_ERR_INVALID_ARG;
+  if (ns_steps < 0 || ns_steps > kMaxSteps) return MUON_ERR_INVALID_ARG;
+  float co[3];
+  rc = check_coeffs(coeffs, co);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) {
+    if (!params[i] || !grads[i] || !bufs[i]) return MUON_ERR_INVALID_ARG;
+    if (!aligned16(params[i]) || !aligned16(grads[i]) || !aligned16(bufs[i]))
+      return MUON_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  rc = get_ctx(&ctx);
+  if (rc) return rc;
+  for (int g0 = 0; g0 < n; g0 += MUON_MAX_GROUP) {
+    const int gn = std::min(MUON_MAX_GROUP, n - g0);
+    rc = step_group(ctx, params + g0, grads + g0, bufs + g0, shapes + 2 * g0, gn, lr, beta, nesterov,
+                    ns_steps, co, static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+  }
+  return MUON_OK;
+}
+
+int muon_orthogonalize(const float* x, void* out, int out_is_bf16, int64_t rows, int64_t cols,
+                       int ns_steps, const float* coeffs, void* stream) {
+  const int64_t shp[2] = {rows, cols};
+  int rc = check_shapes(shp, 1);
+  if (rc) return rc;
+  if (!x || !out) return MUON_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MUON_ERR_UNSUPPORTED;
+  if (ns_steps < 0 || ns_steps > kMaxSteps) return MUON_ERR_INVALID_ARG;
+  float co[3];
+  rc = check_coeffs(coeffs, co);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  rc = get_ctx(&ctx);
+  if (rc) return rc;
+  std::vector<Geom> geom = make_geom(shp, 1);
+  Plan* P = nullptr;
+  rc = get_plan(ctx, shape_key('O', geom), geom, true, &P);
+  if (rc) return rc;
+  K1Ptrs p;
+  p.g = x;
+  p.buf = nullptr;
+  p.x0 = P->X[0];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = run_k1(ctx, P, &p, K1_PLAIN, 0.f, 0, s);
+  if (rc) return rc;
+  const int mode = out_is_bf16 ? FINAL_OUT_BF16 : FINAL_OUT_F32;
+  if (ns_steps == 0) {
+    void* dst[1] = {out};
+    return run_apply(P, mode, dst, nullptr, s);
+  }
+  static thread_local FinalTable F;
+  F.ptr[0] = out;
+  F.scale[0] = 0.f;
+  return run_ns(ctx, P, ns_steps, co, mode, &F, s);
+}
+
+int muon_momentum_normalize(const float* const* grads, float* const* bufs, uint16_t* const* x0,
+                            const int64_t* x0_ld, const int64_t* shapes, int n, float beta,
+                            int nesterov, void* stream) {
+  int rc = check_shapes(shapes, n);
+  if (rc) return rc;
+  if (n == 0) return MUON_OK;
+  if (n > MUON_MAX_GROUP) return MUON_ERR_INVALID_ARG;
+  if (!grads || !bufs || !x0 || !x0_ld || !std::isfinite(beta)) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!grads[i] || !bufs[i] || !x0[i]) return MUON_ERR_INVALID_ARG;
+    if (!aligned16(grads[i]) || !aligned16(bufs[i]) || !aligned16(x0[i])) return MUON_ERR_UNSUPPORTED;
+    const long long ncols = std::max(shapes[2 * i], shapes[2 * i + 1]);
+    if (x0_ld[i] < ncols || (x0_ld[i] & 7)) return MUON_ERR_INVALID_ARG;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  rc = get_ctx(&ctx);
+  if (rc) return rc;
+  std::vector<Geom> geom = make_geom(shapes, n);
+  std::vector<long long> key = shape_key('K', geom);
+  for (int i = 0; i < n; ++i) {
+    geom[i].ldx = x0_ld[i];
+    key.push_back(x0_ld[i]);
+  }
+  Plan* P = nullptr;
+  rc = get_plan(ctx, key, geom, false, &P);
+  if (rc) return rc;
+  std::vector<K1Ptrs> ptrs(n);
+  for (int i = 0; i < n; ++i) {
+    ptrs[i].g = grads[i];
+    ptrs[i].buf = bufs[i];
+    ptrs[i].x0 = reinterpret_cast<__nv_bfloat16*>(x0[i]);
+  }
+  return run_k1(ctx, P, ptrs.data(), K1_MOMENTUM, beta, nesterov, static_cast<cudaStream_t>(stream));
+}
+
+// One GEMM phase on caller buffers (stage entry points).
+static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t* opB, long long ldB,
+                     long long rowsB, long long colsB, const uint16_t* epi, long long ld_epi,
+                     uint16_t* out, long long ld_out, long long M, long long N, long long K, float ca,
+                     float cb, float cc, void* stream) {
+  DeviceCtx* ctx = nullptr;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  std::vector<long long> key = {'G', op, (long long)(uintptr_t)opA, ldA, (long long)(uintptr_t)opB, ldB,
+                                rowsB, colsB, (long long)(uintptr_t)epi, ld_epi,
+                                (long long)(uintptr_t)out, ld_out, M, N, K};
+  Plan* P = nullptr;
+  if (ctx->stage_plans.size() >= 64 && !ctx->stage_plans.count(key)) {
+    // Bounded cache: older stage plans may still be read by queued kernels.
+    if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
+    ctx->stage_plans.clear();
+  }
+  auto it = ctx->stage_plans.find(key);
+  if (it != ctx->stage_plans.end()) {
+    P = it->second.get();
+  } else {
+    std::unique_ptr<Plan> np(new Plan());
+    std::vector<NsTile> tiles;
+    const int kc = (int)cdiv(K, BK);
+    if (op == OP_UPDATE)
+      full_tiles(tiles, 0, M, N, kc);
+    else
+      sym_tiles(tiles, 0, M, kc);
+    const size_t bytes = 256 + sizeof(NsProblem) + sizeof(NsTile) * tiles.size();
+    if (cudaMalloc(&np->mem.ptr, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_NOMEM;
+    }
+    np->mem.bytes = bytes;
+    NsProblem q;
+    std::memset(&q, 0, sizeof(q));
+    if (!make_map(&q.tmA, opA, M, K, ldA)) return MUON_ERR_CUDA;
+    if (!make_map(&q.tmB, opB, rowsB, colsB, ldB)) return MUON_ERR_CUDA;
+    q.epi = reinterpret_cast<const __nv_bfloat16*>(epi);
+    q.ld_epi = ld_epi;
+    q.out = reinterpret_cast<__nv_bfloat16*>(out);
+    q.ld_out = ld_out;
+    q.M = (int)M;
+    q.N = (int)N;
+    q.K = (int)K;
+    std::vector<NsProblem> pr(1, q);
+    rc = upload_phase(np->poly, np->mem.ptr, 0, 256 + sizeof(NsProblem), pr, tiles);
+    if (rc) return rc;
+    P = np.get();
+    ctx->stage_plans[key] = std::move(np);
+  }
+  NsLaunch L;
+  L.probs = P->poly.probs;
+  L.tiles = P->poly.tiles;
+  L.ntiles = P->poly.ntiles;
+  L.final_mode = FINAL_NONE;
+  L.ca = ca;
+  L.cb = cb;
+  L.cc = cc;
+  L.limit_ns = limit_ns();
+  L.status = ctx->status;
+  return cuda_err(launch_ns_gemm(op, L, nullptr, std::min(L.ntiles, ctx->num_sms),
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+static bool ld_ok(long long ld, long long minv) { return ld >= minv && (ld & 7) == 0; }
+
+int muon_gram(const uint16_t* x, int64_t ld_x, uint16_t* a, int64_t ld_a, int64_t m, int64_t n,
+              void* stream) {
+  if (!x || !a || m <= 0 || n <= 0 || !ld_ok(ld_x, n) || !ld_ok(ld_a, m)) return MUON_ERR_INVALID_ARG;
+  if (m >= (1ll << 30) || n >= (1ll << 30)) return MUON_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(a)) return MUON_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return run_stage(OP_GRAM, x, ld_x, x, ld_x, m, n, nullptr, 0, a, ld_a, m, m, n, 0.f, 0.f, 0.f, stream);
+}
+
+int muon_poly(const uint16_t* a, int64_t ld_a, uint16_t* b_out, int64_t ld_b, int64_t m, float cb,
+              float cc, void* stream) {
+  if (!a || !b_out || m <= 0 || !ld_ok(ld_a, m) || !ld_ok(ld_b, m)) return MUON_ERR_INVALID_ARG;
+  if (!std::isfinite(cb) || !std::isfinite(cc)) return MUON_ERR_INVALID_ARG;
+  if (m >= (1ll << 30)) return MUON_ERR_UNSUPPORTED;
+  if (!aligned16(a) || !aligned16(b_out)) return MUON_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return run_stage(OP_POLY, a, ld_a, a, ld_a, m, m, a, ld_a, b_out, ld_b, m, m, m, 0.f, cb, cc, stream);
+}
+
+int muon_xupdate(const uint16_t* b, int64_t ld_b, const uint16_t* x, int64_t ld_x, uint16_t* x_out,
+                 int64_t ld_out, int64_t m, int64_t n, float ca, void* stream) {
+  if (!b || !x || !x_out || m <= 0 || n <= 0) return MUON_ERR_INVALID_ARG;
+  if (!ld_ok(ld_b, m) || !ld_ok(ld_x, n) || !ld_ok(ld_out, n) || !std::isfinite(ca))
+    return MUON_ERR_INVALID_ARG;
+  if (x_out == x) return MUON_ERR_INVALID_ARG;
+  if (m >= (1ll << 30) || n >= (1ll << 30)) return MUON_ERR_UNSUPPORTED;
+  if (!aligned16(b) || !aligned16(x) || !aligned16(x_out)) return MUON_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return run_stage(OP_UPDATE, b, ld_b, x, ld_x, m, n, x, ld_x, x_out, ld_out, m, n, m, ca, 0.f, 0.f,
+                   stream);
+}
+
+int muon_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  int h = 0;
+  if (cudaMemcpy(&h, ctx->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (h != 0 && cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return MUON_ERR_CUDA;
+  return h;
+}
+
+const char* muon_error_string(int code) {
+  switch (code) {
+    case MUON_OK: return "success";
+    case MUON_ERR_INVALID_ARG: return "invalid argument";
+    case MUON_ERR_UNSUPPORTED: return "unsupported (alignment, size or device)";
+    case MUON_ERR_CUDA: return "CUDA error";
+    case MUON_ERR_NOMEM: return "out of device memory";
+    case MUON_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+void muon_set_wait_limit_ns(uint64_t ns) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_limit_from_env = true;
+  g_limit_ns = ns;
+}
+
+int64_t muon_workspace_bytes(const int64_t* shapes, int n) {
+  if (check_shapes(shapes, n)) return -1;
+  int64_t tot = 0;
+  for (int g0 = 0; g0 < n; g0 += MUON_MAX_GROUP) {
+    const int gn = std::min(MUON_MAX_GROUP, n - g0);
+    tot += (int64_t)plan_bytes(make_geom(shapes + 2 * g0, gn), true);
+  }
+  return tot;
+}
+
+void muon_profile_begin(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_prof.on = true;
+}
+
+int muon_profile_end(double* ms, int64_t* launches, int nkinds) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_prof.on = false;
+  if (!ms || !launches || nkinds < 0) return MUON_ERR_INVALID_ARG;
+  for (int k = 0; k < nkinds; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  int rc = MUON_OK;
+  for (const ProfRecord& r : g_prof.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+      rc = MUON_ERR_CUDA;
+    if (r.kind < nkinds) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    g_prof.pool.push_back(r.start);
+    g_prof.pool.push_back(r.stop);
+  }
+  g_prof.recs.clear();
+  return rc ? rc : std::min(nkinds, (int)MUON_PROFILE_KINDS);
+}
+
+void muon_release(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_ctx) {
+    cudaSetDevice(kv.first);
+    cudaDeviceSynchronize();
+    kv.second->plans.clear();
+    kv.second->stage_plans.clear();
+    if (kv.second->status) cudaFree(kv.second->status);
+  }
+  g_ctx.clear();
+  cudaSetDevice(cur);
+}
+
+const char* muon_version(void) { return "muon-b200 0.1 (sm_100a, tcgen05)"; }
+
+}  // extern "C"

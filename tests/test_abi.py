@@ -1,0 +1,92 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+argument checks reject bad input before any GPU work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MUON_API\s+[\w\s\*]*?\b(muon_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from newton_schulz_norm_b200 import build
+    build.build()
+    import newton_schulz_norm_b200 as m
+    return m.library()
+
+
+def test_header_declares_expected_entry_points():
+    syms = _declared_symbols()
+    for s in ("muon_step", "muon_orthogonalize", "muon_status", "muon_error_string",
+              "muon_release", "muon_momentum_normalize", "muon_gram", "muon_poly", "muon_xupdate"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import newton_schulz_norm_b200 as m
+    syms = _declared_symbols()
+    assert sorted(m.EXPORTS) == syms
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_no_cpu_fallback_symbols(lib):
+    # The library is CUDA-only: its entry points are the declared ones, and the
+    # package carries no oracle import.
+    import newton_schulz_norm_b200 as m
+    src = open(m.__file__).read()
+    assert "oracle" not in src.replace("# ", "")
+
+
+def test_version_and_errors(lib):
+    assert b"sm_100a" in lib.muon_version()
+    assert lib.muon_error_string(0) == b"success"
+    assert lib.muon_error_string(-5) == b"device-side wait timed out"
+    assert lib.muon_error_string(12345) == b"unknown status"
+
+
+def test_argument_checks_without_gpu(lib):
+    P = ctypes.c_void_p
+    arr = (P * 1)(P(16))
+    sh = (ctypes.c_int64 * 2)(4, 4)
+    # n = 0 is a no-op
+    assert lib.muon_step(None, None, None, None, 0, 0.1, 0.9, 1, 5, None, None) == 0
+    # negative n, null pointer arrays, bad shapes, bad steps, non-finite scalars
+    assert lib.muon_step(arr, arr, arr, sh, -1, 0.1, 0.9, 1, 5, None, None) == -1
+    assert lib.muon_step(None, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, None) == -1
+    bad = (ctypes.c_int64 * 2)(0, 4)
+    assert lib.muon_step(arr, arr, arr, bad, 1, 0.1, 0.9, 1, 5, None, None) == -1
+    assert lib.muon_step(arr, arr, arr, sh, 1, 0.1, 0.9, 1, -1, None, None) == -1
+    assert lib.muon_step(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 101, None, None) == -1
+    assert lib.muon_step(arr, arr, arr, sh, 1, float("nan"), 0.9, 1, 5, None, None) == -1
+    nanco = (ctypes.c_float * 3)(1.0, float("inf"), 0.0)
+    assert lib.muon_step(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 5, nanco, None) == -1
+    # misaligned device pointer
+    mis = (P * 1)(P(18))
+    assert lib.muon_step(mis, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, None) == -2
+    # oversized matrix
+    big = (ctypes.c_int64 * 2)(1 << 16, 1 << 16)
+    assert lib.muon_step(arr, arr, arr, big, 1, 0.1, 0.9, 1, 5, None, None) == -2
+    # stage entry points
+    assert lib.muon_gram(None, 8, None, 8, 4, 4, None) == -1
+    assert lib.muon_gram(P(16), 6, P(16), 8, 4, 4, None) == -1      # ld not a multiple of 8
+    assert lib.muon_xupdate(P(16), 8, P(32), 8, P(32), 8, 4, 4, 3.0, None) == -1   # aliasing
+    assert lib.muon_orthogonalize(None, None, 0, 4, 4, 5, None, None) == -1
+
+
+def test_workspace_bytes_host_only(lib):
+    import newton_schulz_norm_b200 as m
+    from workloads import WORKLOADS
+    b = m.workspace_bytes(WORKLOADS["gpt2_124m"].shapes)
+    # two bf16 iterates (85M elements each) + A and B (48 x 768^2 each) + small tables
+    lower = 2 * 2 * 84934656 + 2 * 2 * 48 * 768 * 768
+    assert lower <= b <= lower * 1.05
+    assert m.workspace_bytes([(0, 3)]) == -1

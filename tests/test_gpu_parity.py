@@ -1,0 +1,364 @@
+"""GPU parity: every kernel of the Muon step, through the C-ABI, against the
+CPU oracle on the same seeded inputs.
+
+Tolerances (from the arithmetic, stated per check):
+* momentum buffers: both sides do one fp32 rounding of beta*buf + g, so the
+  relative error is at most one fp32 ulp (<= 1.2e-7); the bar is 1e-6.
+* X0: both sides divide the same fp32 u by the norm in (at least) double
+  precision before one bf16 rounding: at most 1 bf16 ulp apart.
+* bf16 GEMM stage outputs (A, B, X1): the GPU accumulates in fp32, the oracle
+  in fp64.  Each difference must stay within 1 bf16 ulp plus the rigorous
+  fp32 accumulation bound 2 K 2^-24 (|P||Q|)_ij of the product P Q (which
+  matters only for entries that cancel to near zero), and differ on at most
+  1% of entries.
+* orthogonalised update X and new parameters: relative Frobenius error
+  <= 1e-2 (five iterations compound the rare 1-ulp differences); the update
+  Delta p is checked at the same bar, since p alone would hide its error.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import (bf16_round, coeffs_f32, momentum_ref, muon_step_ref, newton_schulz_ref,
+                    normalize_ref, orient, orthogonalize_ref)
+from tests.gpu_util import (bf16_agreement, bf16_close, fp32_gemm_bound, rel_fro, to_bf16, to_f32,
+                            to_np)
+from tests.spectral import closed_form_ns, lift_threshold, poly_scalar
+from workloads import WORKLOADS, WorkloadStream, square_case
+
+pytestmark = pytest.mark.gpu
+
+COEFFS = (3.4445, -4.7750, 2.0315)
+X_TOL = 1e-2
+BUF_TOL = 1e-6
+
+
+@pytest.fixture(scope="module")
+def muon():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from newton_schulz_norm_b200 import build
+    build.build()
+    import newton_schulz_norm_b200 as m
+    m.set_wait_limit_ns(2_000_000_000)
+    yield m
+    assert m.status() == 0
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- first kernel
+
+SHAPES_K1 = [(256, 256), (64, 200), (200, 64), (7, 13), (13, 7), (1, 1), (1, 100), (100, 1),
+             (129, 257), (257, 129), (768, 2304), (3072, 768), (65, 66)]
+
+
+@pytest.mark.parametrize("nesterov", [True, False])
+def test_momentum_normalize_stage(muon, nesterov):
+    rng = _rng(1)
+    gs = [rng.standard_normal(s).astype(np.float32) for s in SHAPES_K1]
+    bs = [(rng.standard_normal(s) * 0.1).astype(np.float32) for s in SHAPES_K1]
+    g_d = [to_f32(g) for g in gs]
+    b_d = [to_f32(b) for b in bs]
+    x0_d = muon.momentum_normalize(g_d, b_d, beta=0.95, nesterov=nesterov)
+    torch.cuda.synchronize()
+    assert muon.status() == 0
+    for g, b, bd, xd in zip(gs, bs, b_d, x0_d):
+        buf_ref, u = momentum_ref(g, b, 0.95, nesterov)
+        got = to_np(bd)
+        assert np.max(np.abs(got - buf_ref)) <= BUF_TOL * max(np.max(np.abs(buf_ref)), 1e-30)
+        x0_ref, _ = orient(normalize_ref(u))
+        x0 = to_np(xd)
+        assert x0.shape == x0_ref.shape
+        mism, ulps = bf16_agreement(x0, x0_ref)
+        assert ulps <= 1.0 and mism <= 1e-3, (g.shape, mism, ulps)
+
+
+def test_momentum_three_steps_exact_match(muon):
+    """Hand-worked recurrence (g = 1, beta = 0.95) through the GPU kernel."""
+    g = torch.ones((16, 24), device="cuda")
+    b = torch.zeros((16, 24), device="cuda")
+    expect_buf = [1.0, 1.95, 2.8525]
+    for e in expect_buf:
+        muon.momentum_normalize([g], [b], beta=0.95, nesterov=True)
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(to_np(b), e, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- NS stages
+
+NS_SHAPES = [(7, 20), (64, 64), (128, 256), (200, 333), (256, 1024), (768, 768), (768, 3072),
+             (130, 300), (1, 9)]
+
+
+def _trace_inputs(m, n, seed):
+    rng = _rng(seed)
+    g = rng.standard_normal((m, n))
+    x0 = normalize_ref(g)
+    x1, hist = newton_schulz_ref(x0, 1, COEFFS, trace=True)
+    A, B, X1 = hist[0]
+    return x0, A, B, X1
+
+
+@pytest.mark.parametrize("m,n", NS_SHAPES)
+def test_gram_stage(muon, m, n):
+    x0, A, _, _ = _trace_inputs(m, n, 10 + m)
+    a = to_np(muon.gram(to_bf16(x0)))
+    torch.cuda.synchronize()
+    mism, _ = bf16_agreement(a, A)
+    ratio = bf16_close(a, A, fp32_gemm_bound(x0, x0.T, n))
+    assert ratio <= 1.0 and mism <= 1e-2, (mism, ratio)
+    assert np.array_equal(a, a.T)
+
+
+@pytest.mark.parametrize("m,n", NS_SHAPES)
+def test_poly_stage(muon, m, n):
+    _, A, B, _ = _trace_inputs(m, n, 20 + m)
+    a, b, c = coeffs_f32(COEFFS)
+    out = to_np(muon.poly(to_bf16(A), b, c))
+    torch.cuda.synchronize()
+    mism, _ = bf16_agreement(out, B)
+    # fp32 product A A (m terms) scaled by |c|, plus the fp32 epilogue b*A + c*acc
+    bound = abs(c) * fp32_gemm_bound(A, A, m) + 2.0 ** -22 * (abs(b) * np.abs(A) + abs(c) * (np.abs(A) @ np.abs(A)))
+    ratio = bf16_close(out, B, bound)
+    assert ratio <= 1.0 and mism <= 1e-2, (mism, ratio)
+    assert np.array_equal(out, out.T)
+
+
+@pytest.mark.parametrize("m,n", NS_SHAPES)
+def test_xupdate_stage(muon, m, n):
+    x0, _, B, X1 = _trace_inputs(m, n, 30 + m)
+    a, _, _ = coeffs_f32(COEFFS)
+    out = to_np(muon.xupdate(to_bf16(B), to_bf16(x0), a))
+    torch.cuda.synchronize()
+    mism, _ = bf16_agreement(out, X1)
+    bound = fp32_gemm_bound(B, x0, m) + 2.0 ** -22 * (abs(a) * np.abs(x0) + np.abs(B) @ np.abs(x0))
+    ratio = bf16_close(out, X1, bound)
+    assert ratio <= 1.0 and mism <= 1e-2, (mism, ratio)
+
+
+# ---------------------------------------------------------------- orthogonalize
+
+@pytest.mark.parametrize("shape", [(256, 256), (64, 200), (200, 64), (300, 1000), (1000, 300),
+                                   (5, 5), (1, 33), (33, 1), (768, 3072)])
+@pytest.mark.parametrize("steps", [1, 5])
+def test_orthogonalize_vs_oracle(muon, shape, steps):
+    rng = _rng(40 + shape[0])
+    x = rng.standard_normal(shape).astype(np.float32)
+    ref = orthogonalize_ref(x, steps, COEFFS)
+    out = to_np(muon.orthogonalize(to_f32(x), ns_steps=steps))
+    torch.cuda.synchronize()
+    assert rel_fro(out, ref) <= X_TOL
+    outb = to_np(muon.orthogonalize(to_f32(x), ns_steps=steps, out_dtype=torch.bfloat16))
+    np.testing.assert_array_equal(outb, out)   # fp32 output holds the bf16 values
+
+
+def test_orthogonalize_zero_steps_is_x0(muon):
+    rng = _rng(50)
+    x = rng.standard_normal((40, 96)).astype(np.float32)
+    out = to_np(muon.orthogonalize(to_f32(x), ns_steps=0))
+    mism, ulps = bf16_agreement(out, normalize_ref(x))
+    assert ulps <= 1.0 and mism <= 1e-3
+
+
+def test_orthogonalize_singular_values(muon):
+    """Output singular values: <= 1.2024 + slack always; >= 0.6 for every
+    direction whose normalised input value the closed form lifts above 0.6."""
+    rng = _rng(51)
+    x = rng.standard_normal((256, 256)).astype(np.float32)
+    out = to_np(muon.orthogonalize(to_f32(x), ns_steps=5))
+    sv = np.linalg.svd(out, compute_uv=False)
+    s0 = np.linalg.svd(x / np.linalg.norm(x), compute_uv=False)
+    assert sv.max() <= 1.3
+    thr = lift_threshold(0.6)
+    assert np.sum(sv >= 0.6 - 0.02) >= np.sum(s0 >= thr)
+    # the literal band, reported: most of a Gaussian's spectrum lies in it
+    assert np.mean((sv >= 0.6) & (sv <= 1.3)) > 0.9
+
+
+@pytest.mark.parametrize("n", [1024, 2048])
+def test_square_sweep_vs_oracle(muon, n):
+    case = square_case(n, seed=0)
+    ref = orthogonalize_ref(case.g, 5, COEFFS)
+    out = to_np(muon.orthogonalize(to_f32(case.g), ns_steps=5))
+    assert rel_fro(out, ref) <= X_TOL
+    # closed form through the known factors: U^T X V ~ diag(p^5(sigma/||sigma||))
+    d = case.project(out)
+    target = poly_scalar(case.sigma / np.linalg.norm(case.sigma), COEFFS, 5)
+    assert rel_fro(np.diag(d), target) < 3e-2
+    off = d - np.diag(np.diag(d))
+    assert np.linalg.norm(off) / np.linalg.norm(target) < 5e-2
+
+
+def test_square_4096_closed_form(muon):
+    case = square_case(4096, seed=0)
+    out = to_np(muon.orthogonalize(to_f32(case.g), ns_steps=5))
+    d = case.project(out)
+    target = poly_scalar(case.sigma / np.linalg.norm(case.sigma), COEFFS, 5)
+    assert rel_fro(np.diag(d), target) < 3e-2
+
+
+# ---------------------------------------------------------------- full step
+
+def _run_step(muon, params, grads, bufs, **kw):
+    p_d = [to_f32(p) for p in params]
+    g_d = [to_f32(g) for g in grads]
+    b_d = [to_f32(b) for b in bufs]
+    muon.step(p_d, g_d, b_d, **kw)
+    torch.cuda.synchronize()
+    return p_d, b_d
+
+
+def _check_step(p_old, p_gpu, b_gpu, p_ref, b_ref, tol=X_TOL):
+    for po, pg, bg, pr, br in zip(p_old, p_gpu, b_gpu, p_ref, b_ref):
+        pg = to_np(pg)
+        bg = to_np(bg)
+        assert np.max(np.abs(bg - br)) <= BUF_TOL * max(np.max(np.abs(br)), 1e-30)
+        assert rel_fro(pg, pr) <= tol
+        dp_g = pg - po
+        dp_r = np.asarray(pr, np.float64) - po
+        assert rel_fro(dp_g, dp_r) <= tol, (po.shape, rel_fro(dp_g, dp_r))
+
+
+EDGE_SHAPES = [(1, 1), (1, 100), (100, 1), (7, 13), (13, 7), (64, 64), (129, 257), (257, 129),
+               (300, 1000), (1000, 300)]
+
+
+@pytest.mark.parametrize("steps", [0, 1, 2, 5])
+def test_step_edge_shapes(muon, steps):
+    rng = _rng(60 + steps)
+    ps = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in EDGE_SHAPES]
+    gs = [rng.standard_normal(s).astype(np.float32) for s in EDGE_SHAPES]
+    bs = [(rng.standard_normal(s) * 0.1).astype(np.float32) for s in EDGE_SHAPES]
+    p_d, b_d = _run_step(muon, ps, gs, bs, lr=0.02, ns_steps=steps)
+    p_ref, b_ref = muon_step_ref(ps, gs, bs, lr=0.02, ns_steps=steps)
+    _check_step(ps, p_d, b_d, p_ref, b_ref)
+
+
+def test_step_options(muon):
+    """nesterov off, another coefficient triple, another lr and beta."""
+    rng = _rng(70)
+    shapes = [(96, 160), (160, 96), (128, 128)]
+    ps = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in shapes]
+    gs = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    bs = [(rng.standard_normal(s) * 0.1).astype(np.float32) for s in shapes]
+    co = (1.875, -1.25, 0.375)
+    p_d, b_d = _run_step(muon, ps, gs, bs, lr=0.1, beta=0.9, nesterov=False, ns_steps=4, coeffs=co)
+    p_ref, b_ref = muon_step_ref(ps, gs, bs, lr=0.1, beta=0.9, nesterov=False, ns_steps=4, coeffs=co)
+    _check_step(ps, p_d, b_d, p_ref, b_ref)
+
+
+def test_step_zero_grad_and_nan_isolation(muon):
+    shapes = [(32, 48), (48, 32), (40, 40)]
+    rng = _rng(71)
+    ps = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in shapes]
+    gs = [np.zeros(shapes[0], np.float32), rng.standard_normal(shapes[1]).astype(np.float32),
+          rng.standard_normal(shapes[2]).astype(np.float32)]
+    gs[1][3, 5] = np.nan
+    bs = [np.zeros(s, np.float32) for s in shapes]
+    p_d, b_d = _run_step(muon, ps, gs, bs, lr=0.02)
+    assert np.array_equal(to_np(p_d[0]), ps[0])        # zero update leaves p
+    assert np.isnan(to_np(p_d[1])).any()               # NaN stays in its matrix
+    assert np.isfinite(to_np(p_d[2])).all()
+    p_ref, b_ref = muon_step_ref(ps[2:], gs[2:], bs[2:], lr=0.02)
+    _check_step(ps[2:], p_d[2:], b_d[2:], p_ref, b_ref)
+
+
+@pytest.mark.parametrize("name,steps", [("single_256", 3), ("gpt2_block", 3)])
+def test_step_workloads_consecutive(muon, name, steps):
+    wl = WORKLOADS[name]
+    st = WorkloadStream(wl, seed=0)
+    params, bufs = st.init()
+    p_d = [to_f32(p) for p in params]
+    b_d = [to_f32(b) for b in bufs]
+    p_ref = [p.copy() for p in params]
+    b_ref = [b.copy() for b in bufs]
+    for _ in range(steps):
+        grads = st.next_grads()
+        p_old = [p.copy() for p in p_ref]
+        muon.step(p_d, [to_f32(g) for g in grads], b_d, lr=wl.lr, beta=wl.beta,
+                  nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+        torch.cuda.synchronize()
+        p_ref, b_ref = muon_step_ref(p_ref, grads, b_ref, lr=wl.lr, beta=wl.beta,
+                                     nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+        _check_step(p_old, p_d, b_d, p_ref, b_ref)
+        # keep the two trajectories on the same state, so that each step is
+        # compared from identical inputs
+        for i in range(len(p_d)):
+            p_d[i].copy_(to_f32(p_ref[i]))
+            b_d[i].copy_(to_f32(b_ref[i]))
+    assert muon.status() == 0
+
+
+def test_step_gpt2_124m_full_size_sampled(muon):
+    """All 48 matrices in one call (the benchmarked launch configuration);
+    the oracle recomputes a sample of them (one of each shape and the last)."""
+    wl = WORKLOADS["gpt2_124m"]
+    st = WorkloadStream(wl, seed=0)
+    params, bufs = st.init()
+    grads = st.next_grads()
+    p_d, b_d = _run_step(muon, params, grads, bufs, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov,
+                         ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    assert muon.status() == 0
+    sample = [0, 1, 2, 3, 47]
+    p_ref, b_ref = muon_step_ref([params[i] for i in sample], [grads[i] for i in sample],
+                                 [bufs[i] for i in sample], lr=wl.lr, beta=wl.beta,
+                                 nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    _check_step([params[i] for i in sample], [p_d[i] for i in sample], [b_d[i] for i in sample],
+                p_ref, b_ref)
+    # property at full size: every momentum buffer matches the one-rounding form
+    for i in range(0, 48, 7):
+        br, _ = momentum_ref(grads[i], bufs[i], wl.beta, wl.nesterov)
+        assert np.max(np.abs(to_np(b_d[i]) - br)) <= BUF_TOL * np.max(np.abs(br))
+
+
+def test_update_scale_on_transposed(muon):
+    """c_proj-shaped (tall) matrices get sqrt(rows/cols) = 2 times the step."""
+    rng = _rng(80)
+    g = rng.standard_normal((256, 64)).astype(np.float32)
+    p = np.zeros((256, 64), np.float32)
+    b = np.zeros((256, 64), np.float32)
+    p_d, _ = _run_step(muon, [p], [g], [b], lr=0.5)
+    x = orthogonalize_ref((1 + np.float32(0.95)) * g.astype(np.float64), 5, COEFFS)
+    dp = to_np(p_d[0])
+    assert rel_fro(dp, -1.0 * x) <= X_TOL      # lr * sqrt(256/64) = 0.5 * 2
+
+
+def test_timeout_reports_status_and_context_survives(muon):
+    """A wait limit of 0 makes device-side waits give up: the kernels record
+    MUON_ERR_TIMEOUT and return; the next call with the normal limit works."""
+    wl = WORKLOADS["gpt2_block"]
+    st = WorkloadStream(wl, seed=3)
+    params, bufs = st.init()
+    grads = st.next_grads()
+    seen = 0
+    try:
+        for _ in range(3):
+            muon.set_wait_limit_ns(0)
+            _run_step(muon, params, grads, bufs, lr=0.02)
+            seen = muon.status()
+            if seen != 0:
+                break
+    finally:
+        muon.set_wait_limit_ns(2_000_000_000)
+    assert seen == -5
+    p_d, b_d = _run_step(muon, params, grads, bufs, lr=0.02)
+    assert muon.status() == 0
+    p_ref, b_ref = muon_step_ref(params[1:2], grads[1:2], bufs[1:2], lr=0.02)
+    _check_step(params[1:2], p_d[1:2], b_d[1:2], p_ref, b_ref)
+
+
+def test_rejects_bad_args_before_launch(muon):
+    p = torch.zeros((8, 8), device="cuda")
+    g = torch.ones((8, 8), device="cuda")
+    b = torch.zeros((8, 8), device="cuda")
+    with pytest.raises(muon.MuonError):
+        muon.step([p], [g], [b], lr=float("nan"))
+    assert torch.all(p == 0) and torch.all(b == 0)
+    with pytest.raises(muon.MuonError):
+        muon.step([p], [g], [b], lr=0.1, ns_steps=-1)
+    assert torch.all(b == 0)
