@@ -22,11 +22,15 @@ constexpr int BOX_BYTES = BOX * BOX * 2;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int GEMM_THREADS = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int EPI_THREADS = 128;
+constexpr int EPI_WARPS = 8;                // two warps per TMEM lane quarter
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int GEMM_THREADS = 64 + EPI_THREADS;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators of BN columns
+constexpr int EPI_LD = 40;                  // staging row pitch (bf16): 80 B, conflict-free rows
+constexpr int EPI_STAGE_BYTES = 32 * EPI_LD * 2;   // one 32 x 32 bf16 block per epilogue warp
 constexpr int GEMM_BAR_BYTES = 256;
-constexpr size_t GEMM_SMEM_BYTES = size_t(STAGES) * STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
+constexpr size_t GEMM_SMEM_BYTES =
+    size_t(STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
 
 enum NsOp : int { OP_GRAM = 0, OP_POLY = 1, OP_UPDATE = 2 };
 

@@ -15,8 +15,13 @@
 //              swizzle) into a STAGES-deep ring of shared-memory slices;
 //   warp 1     one thread issues tcgen05.mma (M=128, N=256, K=16, fp32
 //              accumulation in TMEM) and commits slices back to the ring;
-//   warps 2-5  read the accumulator from TMEM (tcgen05.ld), apply the fp32
-//              epilogue and store bf16 (or the fp32 parameter update).
+//   warps 2-9  the epilogue: two warps per TMEM lane quarter, each taking
+//              four 32-column chunks of its 32 rows.  A warp reads its chunk
+//              from TMEM (tcgen05.ld, one row per thread), combines it with
+//              the epilogue input, and moves rows <-> coalesced 32x32 blocks
+//              through a private shared-memory block, so every global load
+//              and store is a full-sector, row-contiguous access.  Epilogue
+//              inputs (X or A) are fetched before the accumulator is ready.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
 // overlap the main loop of the next.  Every wait is bounded.
 #include <cstdio>
@@ -36,6 +41,7 @@ constexpr unsigned long long kDrainLimitNs = 1000000000ull;
 
 constexpr uint32_t kIdescK = idesc_bf16_f32(BM, BN, 0);   // B operand K-major
 constexpr uint32_t kIdescMN = idesc_bf16_f32(BM, BN, 1);  // B operand MN-major
+constexpr int CHUNKS_PER_WARP = BN / 32 / 2;               // 4
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   atomicCAS(status, 0, code);
@@ -46,186 +52,224 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Loads 32 bf16 values at row `row`, columns [col0, col0+32) of a row-major
-// matrix (leading dimension ld) as floats; columns >= N read as 0.
-__device__ __forceinline__ void load_row32(const __nv_bfloat16* base, long long ld, int row,
-                                           int col0, int N, float (&o)[32]) {
-  const __nv_bfloat16* p = base + (long long)row * ld + col0;
-  if (col0 + 32 <= N) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack8(const uint4& w, float* o) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint4 w = __ldg(q + v);
-      uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        o[v * 8 + 2 * t] = bf16_bits_to_float(u[t] & 0xFFFFu);
-        o[v * 8 + 2 * t + 1] = bf16_bits_to_float(u[t] >> 16);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 32; ++c)
-      o[c] = (col0 + c < N) ? __bfloat162float(p[c]) : 0.f;
+  for (int t = 0; t < 4; ++t) {
+    o[2 * t] = bf16_bits_to_float(u[t] & 0xFFFFu);
+    o[2 * t + 1] = bf16_bits_to_float(u[t] >> 16);
   }
 }
 
-template <int OP>
-__device__ __forceinline__ void epilogue_chunk(const NsLaunch& L, const NsProblem& P,
-                                               const FinalTable* F, int row, int col0,
-                                               const uint32_t (&acc)[32]) {
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  uint4 w;
+  w.x = pack_bf16x2(x[0], x[1]);
+  w.y = pack_bf16x2(x[2], x[3]);
+  w.z = pack_bf16x2(x[4], x[5]);
+  w.w = pack_bf16x2(x[6], x[7]);
+  return w;
+}
+
+// Coalesced layout of a 32x32 bf16 block: lane holds row (lane>>2) + 8k,
+// columns (lane&3)*8 .. +7, for k = 0..3 (each instruction covers 8 rows x
+// 64 contiguous bytes).
+__device__ __forceinline__ void load_block(const __nv_bfloat16* src, long long ld, int rbase,
+                                           int col0, int M, int N, int lane, uint4 (&r)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = rbase + (lane >> 2) + 8 * k;
+    const int col = col0 + (lane & 3) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (row < M && col < N) {
+      const __nv_bfloat16* p = src + (long long)row * ld + col;
+      if (col + 8 <= N) {
+        w = __ldg(reinterpret_cast<const uint4*>(p));
+      } else {
+        uint16_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int e = 0; e < 8 && col + e < N; ++e) h[e] = __bfloat16_as_ushort(p[e]);
+        w.x = h[0] | ((uint32_t)h[1] << 16);
+        w.y = h[2] | ((uint32_t)h[3] << 16);
+        w.z = h[4] | ((uint32_t)h[5] << 16);
+        w.w = h[6] | ((uint32_t)h[7] << 16);
+      }
+    }
+    r[k] = w;
+  }
+}
+
+// Coalesced block -> one row per lane (through the warp's staging block).
+__device__ __forceinline__ void block_to_rows(uint16_t* stg, const uint4 (&r)[4], int lane,
+                                              float (&row)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    *reinterpret_cast<uint4*>(stg + ((lane >> 2) + 8 * k) * EPI_LD + (lane & 3) * 8) = r[k];
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    unpack8(*reinterpret_cast<const uint4*>(stg + lane * EPI_LD + q * 8), row + 8 * q);
+  __syncwarp();
+}
+
+// One bf16 row per lane -> staging block (row-major).
+__device__ __forceinline__ void rows_to_stage(uint16_t* stg, const float (&x)[32], int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(stg + lane * EPI_LD + q * 8) = pack8(x + 8 * q);
+  __syncwarp();
+}
+
+// Staging block -> global, coalesced.  Element (r, c) of the block goes to
+// dst[(rbase + r) * ld + col0 + c] when (rbase + r) < M, (col0 + c) < N and,
+// for triangle stores, col0 + c >= rbase + r + tri_shift (tri_shift = 0: on
+// or above the diagonal; 1: strictly above; -1 disables the test).
+__device__ __forceinline__ void stage_to_global(const uint16_t* stg, __nv_bfloat16* dst, long long ld,
+                                                int rbase, int col0, int M, int N, int lane,
+                                                int tri_shift) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = (lane >> 2) + 8 * k;
+    const int c = (lane & 3) * 8;
+    const int grow = rbase + r, gcol = col0 + c;
+    if (grow >= M || gcol >= N) continue;
+    const uint4 w = *reinterpret_cast<const uint4*>(stg + r * EPI_LD + c);
+    __nv_bfloat16* p = dst + (long long)grow * ld + gcol;
+    const bool full = (gcol + 8 <= N) && (tri_shift < 0 || gcol >= grow + tri_shift);
+    if (full) {
+      *reinterpret_cast<uint4*>(p) = w;
+    } else {
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const bool ok = (gcol + e < N) && (tri_shift < 0 || gcol + e >= grow + tri_shift);
+        if (ok) p[e] = __ushort_as_bfloat16((uint16_t)((u[e >> 1] >> (16 * (e & 1))) & 0xFFFFu));
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// One row per lane -> transposed staging block: element (lane, c) is stored
+// at staging (c, lane), so the block then holds rows of the mirror image.
+__device__ __forceinline__ void rows_to_stage_t(uint16_t* stg, const float (&x)[32], int lane) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c) stg[c * EPI_LD + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(x[c]));
+  __syncwarp();
+}
+
+// The final iteration's output: X (bf16-rounded) applied to or written into
+// the caller's buffer, in the stored orientation.
+__device__ __forceinline__ void final_chunk(const NsProblem& P, const FinalTable* F, int mode,
+                                            uint16_t* stg, const float (&xb)[32], int rbase,
+                                            int col0, int lane) {
   const int M = P.M, N = P.N;
-  if (row >= M || col0 >= N) return;
-  float x[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(acc[c]);
-
-  if (OP == OP_POLY) {
-    float a[32];
-    load_row32(P.epi, P.ld_epi, row, col0, N, a);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) x[c] = fmaf(L.cc, x[c], L.cb * a[c]);
-  } else if (OP == OP_UPDATE) {
-    float a[32];
-    load_row32(P.epi, P.ld_epi, row, col0, N, a);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) x[c] = fmaf(L.ca, a[c], x[c]);
-  }
-
-  if (OP == OP_GRAM || OP == OP_POLY) {
-    // Symmetric output: entry (row, col) is owned by the tile computing it
-    // with col >= row; it is stored there and mirrored to (col, row).
-    __nv_bfloat16* out = P.out;
-    const long long ld = P.ld_out;
-    if (col0 >= row && col0 + 32 <= N) {
-      uint4* q = reinterpret_cast<uint4*>(out + (long long)row * ld + col0);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_bf16x2(x[v * 8 + 0], x[v * 8 + 1]);
-        w.y = pack_bf16x2(x[v * 8 + 2], x[v * 8 + 3]);
-        w.z = pack_bf16x2(x[v * 8 + 4], x[v * 8 + 5]);
-        w.w = pack_bf16x2(x[v * 8 + 6], x[v * 8 + 7]);
-        q[v] = w;
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int col = col0 + c;
-        if (col >= row && col < N) out[(long long)row * ld + col] = __float2bfloat16_rn(x[c]);
-      }
-    }
-    // Mirror: lanes hold consecutive rows, so each column's 32 stores are
-    // one contiguous 64-byte segment of row `col`.
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int col = col0 + c;
-      if (col > row && col < N) out[(long long)col * ld + row] = __float2bfloat16_rn(x[c]);
-    }
-    return;
-  }
-
-  // OP_UPDATE
-  if (L.final_mode == FINAL_NONE) {
-    __nv_bfloat16* out = P.out;
-    const long long ld = P.ld_out;
-    if (col0 + 32 <= N) {
-      uint4* q = reinterpret_cast<uint4*>(out + (long long)row * ld + col0);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_bf16x2(x[v * 8 + 0], x[v * 8 + 1]);
-        w.y = pack_bf16x2(x[v * 8 + 2], x[v * 8 + 3]);
-        w.z = pack_bf16x2(x[v * 8 + 4], x[v * 8 + 5]);
-        w.w = pack_bf16x2(x[v * 8 + 6], x[v * 8 + 7]);
-        q[v] = w;
-      }
-    } else {
-      for (int c = 0; c < 32; ++c)
-        if (col0 + c < N) out[(long long)row * ld + col0 + c] = __float2bfloat16_rn(x[c]);
-    }
-    return;
-  }
-
-  // Final iteration: round X to bf16 (its storage precision), then write it
-  // to the caller's buffer in the stored orientation or apply the update.
-  float xb[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) xb[c] = __bfloat162float(__float2bfloat16_rn(x[c]));
   const int slot = P.slot;
   const long long ldf = P.ld_final;
-  const int mode = L.final_mode;
   const float neg_scale = -F->scale[slot];
-  if (!P.transposed) {
-    if (mode == FINAL_OUT_BF16) {
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(F->ptr[slot]) + (long long)row * ldf;
-      for (int c = 0; c < 32; ++c)
-        if (col0 + c < N) o[col0 + c] = __float2bfloat16_rn(xb[c]);
-      return;
-    }
-    float* o = reinterpret_cast<float*>(F->ptr[slot]) + (long long)row * ldf + col0;
-    const bool vec = (col0 + 32 <= N) && ((ldf & 3) == 0);
+  if (P.transposed) {
+    // X(row, col) lands at [col][row]; lanes hold consecutive rows, so each
+    // column is one coalesced 128-byte segment.  Loads are issued together.
+    const int row = rbase + lane;
+    const bool rok = row < M;
     if (mode == FINAL_PARAM) {
-      if (vec) {
-        float4* q = reinterpret_cast<float4*>(o);
+      float* base = reinterpret_cast<float*>(F->ptr[slot]);
+      float pv[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          float4 p = q[v];
-          p.x = fmaf(neg_scale, xb[4 * v + 0], p.x);
-          p.y = fmaf(neg_scale, xb[4 * v + 1], p.y);
-          p.z = fmaf(neg_scale, xb[4 * v + 2], p.z);
-          p.w = fmaf(neg_scale, xb[4 * v + 3], p.w);
-          q[v] = p;
-        }
-      } else {
-        for (int c = 0; c < 32; ++c)
-          if (col0 + c < N) o[c] = fmaf(neg_scale, xb[c], o[c]);
-      }
-    } else {  // FINAL_OUT_F32
-      if (vec) {
-        float4* q = reinterpret_cast<float4*>(o);
+      for (int c = 0; c < 32; ++c)
+        pv[c] = (rok && col0 + c < N) ? base[(long long)(col0 + c) * ldf + row] : 0.f;
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          q[v] = make_float4(xb[4 * v], xb[4 * v + 1], xb[4 * v + 2], xb[4 * v + 3]);
-      } else {
-        for (int c = 0; c < 32; ++c)
-          if (col0 + c < N) o[c] = xb[c];
-      }
+      for (int c = 0; c < 32; ++c)
+        if (rok && col0 + c < N) base[(long long)(col0 + c) * ldf + row] = fmaf(neg_scale, xb[c], pv[c]);
+    } else if (mode == FINAL_OUT_F32) {
+      float* base = reinterpret_cast<float*>(F->ptr[slot]);
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (rok && col0 + c < N) base[(long long)(col0 + c) * ldf + row] = xb[c];
+    } else {
+      __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(F->ptr[slot]);
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (rok && col0 + c < N) base[(long long)(col0 + c) * ldf + row] = __float2bfloat16_rn(xb[c]);
     }
     return;
   }
-  // Transposed target: element (row, col) lands at [col][row]; lanes hold
-  // consecutive rows, so every column is one coalesced 128-byte segment.
-#pragma unroll 4
-  for (int c = 0; c < 32; ++c) {
-    const int col = col0 + c;
-    if (col >= N) break;
-    const long long off = (long long)col * ldf + row;
-    if (mode == FINAL_PARAM) {
-      float* o = reinterpret_cast<float*>(F->ptr[slot]) + off;
-      *o = fmaf(neg_scale, xb[c], *o);
-    } else if (mode == FINAL_OUT_F32) {
-      reinterpret_cast<float*>(F->ptr[slot])[off] = xb[c];
-    } else {
-      reinterpret_cast<__nv_bfloat16*>(F->ptr[slot])[off] = __float2bfloat16_rn(xb[c]);
+  rows_to_stage(stg, xb, lane);
+  if (mode == FINAL_OUT_BF16) {
+    stage_to_global(stg, reinterpret_cast<__nv_bfloat16*>(F->ptr[slot]), ldf, rbase, col0, M, N,
+                    lane, -1);
+    return;
+  }
+  // fp32 target, coalesced: lane handles row (lane>>3) + 4k, columns
+  // (lane&7)*4 .. +3 (each instruction covers 4 rows x 128 contiguous bytes).
+  float* base = reinterpret_cast<float*>(F->ptr[slot]);
+  const bool vec_ok = (ldf & 3) == 0;
+  float4 pv[8];
+  if (mode == FINAL_PARAM) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int grow = rbase + (lane >> 3) + 4 * k, gcol = col0 + (lane & 7) * 4;
+      pv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (grow < M && gcol < N) {
+        const float* p = base + (long long)grow * ldf + gcol;
+        if (vec_ok && gcol + 4 <= N) {
+          pv[k] = *reinterpret_cast<const float4*>(p);
+        } else {
+          pv[k].x = p[0];
+          if (gcol + 1 < N) pv[k].y = p[1];
+          if (gcol + 2 < N) pv[k].z = p[2];
+          if (gcol + 3 < N) pv[k].w = p[3];
+        }
+      }
     }
   }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (lane >> 3) + 4 * k, c = (lane & 7) * 4;
+    const int grow = rbase + r, gcol = col0 + c;
+    if (grow >= M || gcol >= N) continue;
+    const uint2 w = *reinterpret_cast<const uint2*>(stg + r * EPI_LD + c);
+    float x4[4] = {bf16_bits_to_float(w.x & 0xFFFFu), bf16_bits_to_float(w.x >> 16),
+                   bf16_bits_to_float(w.y & 0xFFFFu), bf16_bits_to_float(w.y >> 16)};
+    float4 o;
+    if (mode == FINAL_PARAM) {
+      o.x = fmaf(neg_scale, x4[0], pv[k].x);
+      o.y = fmaf(neg_scale, x4[1], pv[k].y);
+      o.z = fmaf(neg_scale, x4[2], pv[k].z);
+      o.w = fmaf(neg_scale, x4[3], pv[k].w);
+    } else {
+      o = make_float4(x4[0], x4[1], x4[2], x4[3]);
+    }
+    float* p = base + (long long)grow * ldf + gcol;
+    if (vec_ok && gcol + 4 <= N) {
+      *reinterpret_cast<float4*>(p) = o;
+    } else {
+      p[0] = o.x;
+      if (gcol + 1 < N) p[1] = o.y;
+      if (gcol + 2 < N) p[2] = o.z;
+      if (gcol + 3 < N) p[3] = o.w;
+    }
+  }
+  __syncwarp();
 }
 
-template <int OP>
+// FINAL = the last X update (writes through FinalTable instead of the next
+// iterate); it fetches its epilogue input per chunk to leave registers for
+// the fp32 read-modify-write of the parameters.
+template <int OP, bool FINAL>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;     // 128B-swizzle atoms need 1 KB alignment
   uint8_t* gbase = smem_raw + (sbase - raw);
-  const uint32_t bar0 = sbase + STAGES * STAGE_BYTES;
+  uint16_t* epi_stage = reinterpret_cast<uint16_t*>(gbase + STAGES * STAGE_BYTES);
+  const uint32_t bar0 = sbase + STAGES * STAGE_BYTES + EPI_WARPS * EPI_STAGE_BYTES;
   // barrier layout: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES +
+                                                    EPI_WARPS * EPI_STAGE_BYTES + 8 * (2 * STAGES + 5));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -362,26 +406,97 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       if (!mbar_wait(drain_bar, 0, kDrainLimitNs)) record_status(L.status, MUON_ERR_TIMEOUT);
     }
   } else {
-    // -------------------------------------------------- epilogue (warps 2-5)
+    // -------------------------------------------------- epilogue (warps 2-9)
+    const int ew = warp - 2;                    // 0..7
     const int quarter = warp & 3;               // TMEM lanes this warp may access
+    const int half = ew >> 2;                   // which 4 of the 8 column chunks
+    uint16_t* stg = epi_stage + ew * (EPI_STAGE_BYTES / 2);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
       const NsTile tile = L.tiles[t];
       const NsProblem& P = L.probs[tile.prob];
+      const int M = P.M, N = P.N;
+      const int rbase = tile.i0 + quarter * 32;
+      const int cbase = tile.j0 + half * (CHUNKS_PER_WARP * 32);
+      // Epilogue input, fetched before the accumulator is ready.
+      constexpr int NPRE = (OP == OP_GRAM) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
+      uint4 ein[NPRE > 0 ? NPRE : 1][4];
+#pragma unroll
+      for (int cc = 0; cc < NPRE; ++cc)
+        load_block(P.epi, P.ld_epi, rbase, cbase + cc * 32, M, N, lane, ein[cc]);
       if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
         record_status(L.status, MUON_ERR_TIMEOUT);
         break;
       }
       tc_fence_after_sync();
-      const int row = tile.i0 + quarter * 32 + lane;
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
+                             half * (CHUNKS_PER_WARP * 32);
+      const bool rows_live = rbase < M;
+      constexpr int UNROLL = FINAL ? 1 : CHUNKS_PER_WARP;
+#pragma unroll UNROLL
+      for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
+        const int col0 = cbase + cc * 32;
+        // the final kernel keeps one chunk of input in flight: fetch chunk cc
+        // (the first was fetched before the wait) while this one is combined
+        uint4 (&ecur)[4] = ein[FINAL ? 0 : (NPRE > 0 ? cc : 0)];
+        if (FINAL && cc > 0) load_block(P.epi, P.ld_epi, rbase, col0, M, N, lane, ecur);
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + ch * 32, v);
+        tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_ld_wait();
-        epilogue_chunk<OP>(L, P, F, row, tile.j0 + ch * 32, v);
+        if (!rows_live || col0 >= N) continue;     // warp-uniform
+        float x[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(v[c]);
+        if (OP == OP_GRAM || OP == OP_POLY) {
+          if (OP == OP_POLY) {
+            float a[32];
+            block_to_rows(stg, ecur, lane, a);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) x[c] = fmaf(L.cc, x[c], L.cb * a[c]);
+          }
+          // Symmetric output: entry (r, c) with c >= r is owned by this tile;
+          // store it and mirror it to (c, r).  Chunks entirely below the
+          // diagonal of this warp's rows are skipped.
+          if (col0 + 31 < rbase) continue;
+          rows_to_stage(stg, x, lane);
+          stage_to_global(stg, P.out, P.ld_out, rbase, col0, M, N, lane, 0);
+          rows_to_stage_t(stg, x, lane);
+          // mirror block: rows col0.., columns rbase..; keep c' > r' there,
+          // i.e. (mirror row) > (mirror column)  <=>  column <= row - 1.
+          for (int k = 0; k < 4; ++k) {
+            const int r = (lane >> 2) + 8 * k;        // mirror row offset (a column of x)
+            const int c = (lane & 3) * 8;             // mirror column offset (a row of x)
+            const int grow = col0 + r, gcol = rbase + c;
+            if (grow >= N || gcol >= M) continue;
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * EPI_LD + c);
+            __nv_bfloat16* p = P.out + (long long)grow * P.ld_out + gcol;
+            if (gcol + 7 < grow && gcol + 8 <= M) {
+              *reinterpret_cast<uint4*>(p) = w;
+            } else {
+              const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if (gcol + e < M && gcol + e < grow)
+                  p[e] = __ushort_as_bfloat16((uint16_t)((u[e >> 1] >> (16 * (e & 1))) & 0xFFFFu));
+            }
+          }
+          __syncwarp();
+        } else {
+          float a[32];
+          block_to_rows(stg, ecur, lane, a);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = fmaf(L.ca, a[c], x[c]);
+          if (!FINAL) {
+            rows_to_stage(stg, x, lane);
+            stage_to_global(stg, P.out, P.ld_out, rbase, col0, M, N, lane, -1);
+          } else {
+            float xb[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) xb[c] = __bfloat162float(__float2bfloat16_rn(x[c]));
+            final_chunk(P, F, L.final_mode, stg, xb, rbase, col0, lane);
+          }
+        }
       }
       tc_fence_before_sync();
       mbar_arrive(tempty_bar(acc));
@@ -403,12 +518,12 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 
 template <int OP>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
-  ns_gemm_body<OP>(L, nullptr);
+  ns_gemm_body<OP, false>(L, nullptr);
 }
 
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     ns_gemm_final_kernel(const __grid_constant__ NsLaunch L, const __grid_constant__ FinalTable F) {
-  ns_gemm_body<OP_UPDATE>(L, &F);
+  ns_gemm_body<OP_UPDATE, true>(L, &F);
 }
 
 }  // namespace
