@@ -26,8 +26,10 @@ constexpr int EPI_WARPS = 8;                // two warps per TMEM lane quarter
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int GEMM_THREADS = 64 + EPI_THREADS;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators of BN columns
-constexpr int EPI_LD = 40;                  // staging row pitch (bf16): 80 B, conflict-free rows
-constexpr int EPI_STAGE_BYTES = 32 * EPI_LD * 2;   // one 32 x 32 bf16 block per epilogue warp
+constexpr int EPI_LD = 40;                  // padded staging pitch (bf16) of the final kernel
+constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;       // one 32 x 32 bf16 block, 64-byte swizzled
+constexpr int EPI_STAGE_BYTES = 2 * EPI_BLOCK_BYTES;   // two blocks per epilogue warp
+constexpr int OUT_BOX = 32;                 // TMA store box: 32 x 32 bf16, 64-byte swizzle
 constexpr int GEMM_BAR_BYTES = 256;
 constexpr size_t GEMM_SMEM_BYTES =
     size_t(STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
@@ -47,6 +49,7 @@ enum FinalMode : int {
 struct alignas(64) NsProblem {
   CUtensorMap tmA;            // A operand source: K-major rows x K
   CUtensorMap tmB;            // B operand source: K-major (Gram, poly) or MN-major (update)
+  CUtensorMap tmOut;          // bf16 output, 32 x 32 boxes, 64-byte swizzle (TMA stores)
   const __nv_bfloat16* epi;   // poly: A (for b*A); update: X (for a*X)
   __nv_bfloat16* out;         // bf16 output (A, B or X_{k+1})
   long long ld_epi;
@@ -85,6 +88,7 @@ struct NsLaunch {
 // 64 x 64 tiles of the stored matrix, in two passes joined per matrix.
 constexpr int K1_TILE = 64;
 constexpr int K1_THREADS = 256;
+constexpr int K1_GROUP = 4;  // 64x64 tiles per work item (one norm partial, one fence)
 
 enum K1Mode : int { K1_MOMENTUM = 0, K1_PLAIN = 1 };
 
@@ -93,7 +97,8 @@ struct K1Info {              // static per matrix (device memory)
   long long ldx;             // leading dimension of the oriented bf16 X0
   int tiles_c;               // tiles along the stored columns
   int ntiles;                // tiles of this matrix
-  int part0;                 // offset of its partial sums
+  int nitems;                // work items of this matrix (groups of K1_GROUP tiles)
+  int part0;                 // offset of its partial sums (one per item)
   int transposed;            // r > c
 };
 
@@ -107,7 +112,7 @@ struct K1Ptrs {              // per call
 // too small for big matrices, so items are two ints.
 struct K1Item {
   int mat;                   // matrix index; pass 2 items have mat | 0x40000000
-  int tile;
+  int group;                 // tiles [group * K1_GROUP, +K1_GROUP) of the matrix
 };
 constexpr int K1_PASS2 = 0x40000000;
 
@@ -143,6 +148,7 @@ cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int g
                            cudaStream_t stream);
 cudaError_t ns_gemm_setup(int device);
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);
+int k1_blocks_per_sm();
 cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream);
 
 }  // namespace muon

@@ -53,7 +53,149 @@ __device__ __forceinline__ float u_from(float g, float bnew, float beta, int mod
   return nesterov ? fmaf(beta, bnew, g) : bnew;
 }
 
-__global__ void __launch_bounds__(K1_THREADS) k1_kernel(const __grid_constant__ K1Launch L) {
+// Pass 1 on one 64 x 64 tile: momentum (buf written back) and this thread's
+// sum of squares of u.  Every load of the thread is issued before any store.
+__device__ __forceinline__ double pass1_tile(const K1Launch& L, const K1Ptrs& P, long long r,
+                                             long long c, long long r0, long long c0, int lrow,
+                                             int lcol) {
+  const bool vec = (c & 3) == 0;
+  const float beta = L.beta;
+  double ss = 0.0;
+  float4 g4[4], b4[4];
+  bool full[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const long long gr = r0 + lrow + 16 * k;
+    const long long gc = c0 + lcol;
+    full[k] = vec && gr < r && gc + 4 <= c;
+    g4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    b4[k] = g4[k];
+    if (full[k]) {
+      const long long off = gr * c + gc;
+      g4[k] = __ldg(reinterpret_cast<const float4*>(P.g + off));
+      if (L.mode != K1_PLAIN) b4[k] = *reinterpret_cast<const float4*>(P.buf + off);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const long long gr = r0 + lrow + 16 * k;
+    const long long gc = c0 + lcol;
+    if (full[k]) {
+      float gv[4] = {g4[k].x, g4[k].y, g4[k].z, g4[k].w};
+      float bv[4] = {b4[k].x, b4[k].y, b4[k].z, b4[k].w};
+      float sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float u = momentum_u(gv[e], bv[e], beta, L.mode, L.nesterov);
+        sq = fmaf(u, u, sq);
+      }
+      ss += (double)sq;
+      if (L.mode != K1_PLAIN)
+        *reinterpret_cast<float4*>(P.buf + gr * c + gc) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    } else if (gr < r && gc < c) {
+      const long long off = gr * c + gc;
+      for (int e = 0; e < 4 && gc + e < c; ++e) {
+        float b = (L.mode != K1_PLAIN) ? P.buf[off + e] : 0.f;
+        const float u = momentum_u(P.g[off + e], b, beta, L.mode, L.nesterov);
+        ss += (double)u * (double)u;
+        if (L.mode != K1_PLAIN) P.buf[off + e] = b;
+      }
+    }
+  }
+  return ss;
+}
+
+// Pass 2 on one 64 x 64 tile: recompute u from g and the new buf, scale by
+// 1/(norm + eps) in double, round once to bf16 and store oriented.
+__device__ __forceinline__ void pass2_tile(const K1Launch& L, const K1Ptrs& P, const K1Info& info,
+                                           long long r0, long long c0, double inv, int tid,
+                                           int lrow, int lcol, uint16_t (*s_tile)[K1_TILE + 2]) {
+  const long long r = info.r, c = info.c;
+  const bool vec = (c & 3) == 0;
+  const float beta = L.beta;
+  const bool tr = info.transposed != 0;
+  float4 g4[4], b4[4];
+  bool full[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const long long gr = r0 + lrow + 16 * k;
+    const long long gc = c0 + lcol;
+    full[k] = vec && gr < r && gc + 4 <= c;
+    g4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    b4[k] = g4[k];
+    if (full[k]) {
+      const long long off = gr * c + gc;
+      g4[k] = __ldg(reinterpret_cast<const float4*>(P.g + off));
+      if (L.mode != K1_PLAIN) b4[k] = __ldcg(reinterpret_cast<const float4*>(P.buf + off));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = lrow + 16 * k;
+    const long long gr = r0 + row;
+    const long long gc = c0 + lcol;
+    uint16_t bits[4] = {0, 0, 0, 0};
+    if (gr < r && gc < c) {
+      const long long off = gr * c + gc;
+      if (full[k]) {
+        const float gv[4] = {g4[k].x, g4[k].y, g4[k].z, g4[k].w};
+        const float bv[4] = {b4[k].x, b4[k].y, b4[k].z, b4[k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float u = u_from(gv[e], bv[e], beta, L.mode, L.nesterov);
+          bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
+        }
+      } else {
+        for (int e = 0; e < 4 && gc + e < c; ++e) {
+          const float b = (L.mode != K1_PLAIN) ? __ldcg(P.buf + off + e) : 0.f;
+          const float u = u_from(P.g[off + e], b, beta, L.mode, L.nesterov);
+          bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
+        }
+      }
+      if (!tr) {
+        __nv_bfloat16* dst = P.x0 + gr * info.ldx + gc;
+        if (gc + 4 <= c) {
+          uint2 w;
+          w.x = (uint32_t)bits[0] | ((uint32_t)bits[1] << 16);
+          w.y = (uint32_t)bits[2] | ((uint32_t)bits[3] << 16);
+          *reinterpret_cast<uint2*>(dst) = w;
+        } else {
+          for (int e = 0; e < 4 && gc + e < c; ++e) dst[e] = __ushort_as_bfloat16(bits[e]);
+        }
+      }
+    }
+    if (tr) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s_tile[row][lcol + e] = bits[e];
+    }
+  }
+  if (tr) {
+    __syncthreads();
+    // X0 row (c0 + oc) holds stored column c0 + oc; 8 threads per row.
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+      const int oc = (tid >> 3) + 32 * k2;
+      const int seg = (tid & 7) * 8;
+      const long long xr = c0 + oc;     // row of X0 (= stored column)
+      const long long xc = r0 + seg;    // first column of X0 (= stored row)
+      if (xr >= c || xc >= r) continue;
+      __nv_bfloat16* dst = P.x0 + xr * info.ldx + xc;
+      if (xc + 8 <= r) {
+        uint4 w;
+        w.x = (uint32_t)s_tile[seg + 0][oc] | ((uint32_t)s_tile[seg + 1][oc] << 16);
+        w.y = (uint32_t)s_tile[seg + 2][oc] | ((uint32_t)s_tile[seg + 3][oc] << 16);
+        w.z = (uint32_t)s_tile[seg + 4][oc] | ((uint32_t)s_tile[seg + 5][oc] << 16);
+        w.w = (uint32_t)s_tile[seg + 6][oc] | ((uint32_t)s_tile[seg + 7][oc] << 16);
+        *reinterpret_cast<uint4*>(dst) = w;
+      } else {
+        for (int e = 0; e < 8 && xc + e < r; ++e) dst[e] = __ushort_as_bfloat16(s_tile[seg + e][oc]);
+      }
+    }
+    __syncthreads();   // s_tile is rewritten by the next tile
+  }
+}
+
+__global__ void __launch_bounds__(K1_THREADS, 4) k1_kernel(const __grid_constant__ K1Launch L) {
   __shared__ int s_item;
   __shared__ int s_flag;
   __shared__ double s_norm;
@@ -75,60 +217,31 @@ __global__ void __launch_bounds__(K1_THREADS) k1_kernel(const __grid_constant__ 
     const int mat = item.mat & ~K1_PASS2;
     const K1Info info = L.info[mat];
     const K1Ptrs P = L.ptrs[mat];
-    const long long r = info.r, c = info.c;
-    const long long r0 = (long long)(item.tile / info.tiles_c) * K1_TILE;
-    const long long c0 = (long long)(item.tile % info.tiles_c) * K1_TILE;
-    const bool vec = (c & 3) == 0;
-    const float beta = L.beta;
+    const int t0 = item.group * K1_GROUP;
+    const int t1 = min(t0 + K1_GROUP, info.ntiles);
 
     if (!pass2) {
       double ss = 0.0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const long long gr = r0 + lrow + 16 * k;
-        const long long gc = c0 + lcol;
-        if (gr >= r || gc >= c) continue;
-        const long long off = gr * c + gc;
-        if (vec && gc + 4 <= c) {
-          const float4 g4 = __ldg(reinterpret_cast<const float4*>(P.g + off));
-          float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-          float bv[4] = {0.f, 0.f, 0.f, 0.f};
-          float4 b4;
-          if (L.mode != K1_PLAIN) {
-            b4 = *reinterpret_cast<const float4*>(P.buf + off);
-            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
-          }
-          float s = 0.f;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float u = momentum_u(gv[e], bv[e], beta, L.mode, L.nesterov);
-            s = fmaf(u, u, s);
-          }
-          ss += (double)s;
-          if (L.mode != K1_PLAIN)
-            *reinterpret_cast<float4*>(P.buf + off) = make_float4(bv[0], bv[1], bv[2], bv[3]);
-        } else {
-          for (int e = 0; e < 4 && gc + e < c; ++e) {
-            float b = (L.mode != K1_PLAIN) ? P.buf[off + e] : 0.f;
-            const float u = momentum_u(P.g[off + e], b, beta, L.mode, L.nesterov);
-            ss += (double)u * (double)u;
-            if (L.mode != K1_PLAIN) P.buf[off + e] = b;
-          }
-        }
+      for (int t = t0; t < t1; ++t) {
+        const long long r0 = (long long)(t / info.tiles_c) * K1_TILE;
+        const long long c0 = (long long)(t % info.tiles_c) * K1_TILE;
+        ss += pass1_tile(L, P, info.r, info.c, r0, c0, lrow, lcol);
       }
       const double tot = block_sum(ss, s_red);
       if (tid == 0) {
-        L.partials[info.part0 + item.tile] = tot;
+        L.partials[info.part0 + item.group] = tot;
+        // Release: this CTA's buf stores (ordered before by the barriers in
+        // block_sum) and the partial become visible before the count does.
         __threadfence();
         const int prev = atomicAdd(L.done + mat, 1);
-        s_flag = (prev == info.ntiles - 1);
+        s_flag = (prev == info.nitems - 1);
       }
       __syncthreads();
       if (s_flag) {
-        // Last tile of this matrix: fixed-order sum of its partials.
+        // Last item of this matrix: fixed-order sum of its partials.
         __threadfence();
         double acc = 0.0;
-        for (int t = tid; t < info.ntiles; t += K1_THREADS) acc += __ldcg(L.partials + info.part0 + t);
+        for (int t = tid; t < info.nitems; t += K1_THREADS) acc += __ldcg(L.partials + info.part0 + t);
         const double all = block_sum(acc, s_red);
         if (tid == 0) {
           L.norms[mat] = sqrt(all);
@@ -143,9 +256,9 @@ __global__ void __launch_bounds__(K1_THREADS) k1_kernel(const __grid_constant__ 
     if (tid == 0) {
       int ok = ld_acquire_gpu(L.ready + mat);
       if (!ok) {
-        const uint64_t t0 = global_timer_ns();
+        const uint64_t t0ns = global_timer_ns();
         while (!(ok = ld_acquire_gpu(L.ready + mat))) {
-          if (global_timer_ns() - t0 > L.limit_ns) break;
+          if (global_timer_ns() - t0ns > L.limit_ns) break;
           __nanosleep(128);
         }
       }
@@ -156,72 +269,10 @@ __global__ void __launch_bounds__(K1_THREADS) k1_kernel(const __grid_constant__ 
     __syncthreads();
     if (!s_flag) continue;
     const double inv = 1.0 / (s_norm + 1e-7);
-    const bool tr = info.transposed != 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int row = lrow + 16 * k;
-      const long long gr = r0 + row;
-      const long long gc = c0 + lcol;
-      uint16_t bits[4] = {0, 0, 0, 0};
-      if (gr < r && gc < c) {
-        const long long off = gr * c + gc;
-        if (vec && gc + 4 <= c) {
-          const float4 g4 = __ldg(reinterpret_cast<const float4*>(P.g + off));
-          float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (L.mode != K1_PLAIN) b4 = __ldcg(reinterpret_cast<const float4*>(P.buf + off));
-          const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float u = u_from(gv[e], bv[e], beta, L.mode, L.nesterov);
-            bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
-          }
-        } else {
-          for (int e = 0; e < 4 && gc + e < c; ++e) {
-            const float b = (L.mode != K1_PLAIN) ? __ldcg(P.buf + off + e) : 0.f;
-            const float u = u_from(P.g[off + e], b, beta, L.mode, L.nesterov);
-            bits[e] = __bfloat16_as_ushort(__double2bfloat16((double)u * inv));
-          }
-        }
-        if (!tr) {
-          __nv_bfloat16* dst = P.x0 + gr * info.ldx + gc;
-          if (gc + 4 <= c) {
-            uint2 w;
-            w.x = (uint32_t)bits[0] | ((uint32_t)bits[1] << 16);
-            w.y = (uint32_t)bits[2] | ((uint32_t)bits[3] << 16);
-            *reinterpret_cast<uint2*>(dst) = w;
-          } else {
-            for (int e = 0; e < 4 && gc + e < c; ++e) dst[e] = __ushort_as_bfloat16(bits[e]);
-          }
-        }
-      }
-      if (tr) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s_tile[row][lcol + e] = bits[e];
-      }
-    }
-    if (tr) {
-      __syncthreads();
-      // X0 row (c0 + oc) holds stored column c0 + oc; 8 threads per row.
-#pragma unroll
-      for (int k2 = 0; k2 < 2; ++k2) {
-        const int oc = (tid >> 3) + 32 * k2;
-        const int seg = (tid & 7) * 8;
-        const long long xr = c0 + oc;     // row of X0 (= stored column)
-        const long long xc = r0 + seg;    // first column of X0 (= stored row)
-        if (xr >= c || xc >= r) continue;
-        __nv_bfloat16* dst = P.x0 + xr * info.ldx + xc;
-        if (xc + 8 <= r) {
-          uint4 w;
-          w.x = (uint32_t)s_tile[seg + 0][oc] | ((uint32_t)s_tile[seg + 1][oc] << 16);
-          w.y = (uint32_t)s_tile[seg + 2][oc] | ((uint32_t)s_tile[seg + 3][oc] << 16);
-          w.z = (uint32_t)s_tile[seg + 4][oc] | ((uint32_t)s_tile[seg + 5][oc] << 16);
-          w.w = (uint32_t)s_tile[seg + 6][oc] | ((uint32_t)s_tile[seg + 7][oc] << 16);
-          *reinterpret_cast<uint4*>(dst) = w;
-        } else {
-          for (int e = 0; e < 8 && xc + e < r; ++e) dst[e] = __ushort_as_bfloat16(s_tile[seg + e][oc]);
-        }
-      }
+    for (int t = t0; t < t1; ++t) {
+      const long long r0 = (long long)(t / info.tiles_c) * K1_TILE;
+      const long long c0 = (long long)(t % info.tiles_c) * K1_TILE;
+      pass2_tile(L, P, info, r0, c0, inv, tid, lrow, lcol, s_tile);
     }
   }
 }
@@ -250,6 +301,13 @@ __global__ void apply_kernel(const __grid_constant__ ApplyLaunch L) {
 }
 
 }  // namespace
+
+int k1_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k1_kernel, K1_THREADS, 0) != cudaSuccess || n < 1)
+    return 1;
+  return n;
+}
 
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream) {
   if (L.nitems <= 0) return cudaSuccess;

@@ -70,6 +70,21 @@ bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols
   return r == CUDA_SUCCESS;
 }
 
+// Output map for TMA stores: 32 x 32 bf16 boxes with 64-byte swizzle (the
+// layout of the epilogue's staging blocks).
+bool make_out_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)OUT_BOX, (cuuint32_t)OUT_BOX};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- device memory arena
 
 struct Arena {
@@ -201,7 +216,7 @@ int get_ctx(DeviceCtx** out) {
   if (cudaMalloc(&ctx->status, sizeof(int)) != cudaSuccess) return MUON_ERR_NOMEM;
   if (cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return MUON_ERR_CUDA;
   if (ns_gemm_setup(dev) != cudaSuccess) return MUON_ERR_CUDA;
-  ctx->k1_blocks_per_sm = 4;
+  ctx->k1_blocks_per_sm = k1_blocks_per_sm();   // persistent: as many CTAs as fit
   *out = ctx.get();
   g_ctx[dev] = std::move(ctx);
   return MUON_OK;
@@ -232,10 +247,10 @@ void full_tiles(std::vector<NsTile>& t, int prob, long long m, long long n, int 
 void k1_items(std::vector<K1Item>& items, const std::vector<K1Info>& info) {
   const int n = (int)info.size();
   auto p1 = [&](int i) {
-    for (int t = 0; t < info[i].ntiles; ++t) items.push_back({i, t});
+    for (int t = 0; t < info[i].nitems; ++t) items.push_back({i, t});
   };
   auto p2 = [&](int i) {
-    for (int t = 0; t < info[i].ntiles; ++t) items.push_back({i | K1_PASS2, t});
+    for (int t = 0; t < info[i].nitems; ++t) items.push_back({i | K1_PASS2, t});
   };
   if (n == 0) return;
   p1(0);
@@ -256,9 +271,10 @@ std::vector<K1Info> k1_infos(const std::vector<Geom>& geom, const std::vector<lo
     k.ldx = ldx[i];
     k.tiles_c = (int)cdiv(k.c, K1_TILE);
     k.ntiles = (int)(cdiv(k.r, K1_TILE) * k.tiles_c);
+    k.nitems = (int)cdiv(k.ntiles, K1_GROUP);
     k.part0 = part;
     k.transposed = geom[i].transposed;
-    part += k.ntiles;
+    part += k.nitems;
     info.push_back(k);
   }
   return info;
@@ -401,6 +417,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan
         q.tmB = q.tmA;
         q.out = P->A + P->a_off[i];
         q.ld_out = g.lda;
+        if (!make_out_map(&q.tmOut, q.out, g.m, g.m, g.lda)) return MUON_ERR_CUDA;
         q.M = (int)g.m;
         q.N = (int)g.m;
         q.K = (int)g.n;
@@ -420,6 +437,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan
         q.ld_epi = g.ldx;
         q.out = P->X[1 - par] + P->x_off[i];
         q.ld_out = g.ldx;
+        if (!make_out_map(&q.tmOut, q.out, g.m, g.n, g.ldx)) return MUON_ERR_CUDA;
         q.M = (int)g.m;
         q.N = (int)g.n;
         q.K = (int)g.m;
@@ -442,6 +460,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan
       q.ld_epi = g.lda;
       q.out = P->B + P->a_off[i];
       q.ld_out = g.lda;
+      if (!make_out_map(&q.tmOut, q.out, g.m, g.m, g.lda)) return MUON_ERR_CUDA;
       q.M = (int)g.m;
       q.N = (int)g.m;
       q.K = (int)g.m;
@@ -781,6 +800,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
     q.ld_epi = ld_epi;
     q.out = reinterpret_cast<__nv_bfloat16*>(out);
     q.ld_out = ld_out;
+    if (!make_out_map(&q.tmOut, out, M, N, ld_out)) return MUON_ERR_CUDA;
     q.M = (int)M;
     q.N = (int)N;
     q.K = (int)K;

@@ -70,6 +70,63 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
   return w;
 }
 
+// This lane's row of the epilogue input: 32 bf16 at (row, col0 .. col0+31)
+// as four 16-byte loads (zeros outside the matrix).
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, long long ld, int row, int col0,
+                                         int M, int N, uint4 (&r)[4]) {
+  const __nv_bfloat16* p = src + (long long)row * ld + col0;
+  if (row < M && col0 + 32 <= N) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = __ldg(reinterpret_cast<const uint4*>(p) + q);
+    return;
+  }
+  uint16_t h[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) h[e] = (row < M && col0 + e < N) ? __bfloat16_as_ushort(p[e]) : 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    r[q].x = h[8 * q + 0] | ((uint32_t)h[8 * q + 1] << 16);
+    r[q].y = h[8 * q + 2] | ((uint32_t)h[8 * q + 3] << 16);
+    r[q].z = h[8 * q + 4] | ((uint32_t)h[8 * q + 5] << 16);
+    r[q].w = h[8 * q + 6] | ((uint32_t)h[8 * q + 7] << 16);
+  }
+}
+
+// A 32 x 32 bf16 staging block in the TMA 64-byte-swizzle layout: row r
+// occupies bytes [64 r, 64 r + 64) and its 16-byte chunk q sits at chunk
+// position q ^ ((r >> 1) & 3).  Row-per-lane writes are bank-conflict free.
+__device__ __forceinline__ uint32_t sw64(int r, int q) {
+  return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void row_to_block(uint8_t* blk, int lane, const float (&x)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(blk + sw64(lane, q)) = pack8(x + 8 * q);
+}
+
+// The lane's 32 values become column `lane` of the block (the mirror image).
+__device__ __forceinline__ void col_to_block(uint8_t* blk, int lane, const float (&x)[32]) {
+  const int q = lane >> 3, e = lane & 7;
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    *reinterpret_cast<uint16_t*>(blk + sw64(c, q) + 2 * e) =
+        __bfloat16_as_ushort(__float2bfloat16_rn(x[c]));
+}
+
+// Diagonal block: entries below the diagonal take the value computed above
+// it, so the stored block is exactly symmetric.  Reads touch only entries
+// above the diagonal and writes only entries below it.
+__device__ __forceinline__ void symmetrize_block(uint8_t* blk, int lane) {
+  const int r = lane;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    if (c < r) {
+      const uint16_t v = *reinterpret_cast<const uint16_t*>(blk + sw64(c, r >> 3) + 2 * (r & 7));
+      *reinterpret_cast<uint16_t*>(blk + sw64(r, c >> 3) + 2 * (c & 7)) = v;
+    }
+  }
+}
+
 // Coalesced layout of a 32x32 bf16 block: lane holds row (lane>>2) + 8k,
 // columns (lane&3)*8 .. +7, for k = 0..3 (each instruction covers 8 rows x
 // 64 contiguous bytes).
@@ -410,7 +467,9 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     const int ew = warp - 2;                    // 0..7
     const int quarter = warp & 3;               // TMEM lanes this warp may access
     const int half = ew >> 2;                   // which 4 of the 8 column chunks
-    uint16_t* stg = epi_stage + ew * (EPI_STAGE_BYTES / 2);
+    uint8_t* stg8 = gbase + STAGES * STAGE_BYTES + ew * EPI_STAGE_BYTES;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(stg8);
+    const uint32_t stg_s = smem_addr(stg8);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
@@ -418,13 +477,13 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       const NsProblem& P = L.probs[tile.prob];
       const int M = P.M, N = P.N;
       const int rbase = tile.i0 + quarter * 32;
+      const int row = rbase + lane;
       const int cbase = tile.j0 + half * (CHUNKS_PER_WARP * 32);
-      // Epilogue input, fetched before the accumulator is ready.
+      // Epilogue input (this lane's row), fetched before the accumulator is ready.
       constexpr int NPRE = (OP == OP_GRAM) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
       uint4 ein[NPRE > 0 ? NPRE : 1][4];
 #pragma unroll
-      for (int cc = 0; cc < NPRE; ++cc)
-        load_block(P.epi, P.ld_epi, rbase, cbase + cc * 32, M, N, lane, ein[cc]);
+      for (int cc = 0; cc < NPRE; ++cc) load_row(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
       if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
         record_status(L.status, MUON_ERR_TIMEOUT);
         break;
@@ -437,10 +496,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 #pragma unroll UNROLL
       for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
         const int col0 = cbase + cc * 32;
-        // the final kernel keeps one chunk of input in flight: fetch chunk cc
-        // (the first was fetched before the wait) while this one is combined
         uint4 (&ecur)[4] = ein[FINAL ? 0 : (NPRE > 0 ? cc : 0)];
-        if (FINAL && cc > 0) load_block(P.epi, P.ld_epi, rbase, col0, M, N, lane, ecur);
+        if (FINAL && cc > 0) load_row(P.epi, P.ld_epi, row, col0, M, N, ecur);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_ld_wait();
@@ -448,54 +505,55 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         float x[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(v[c]);
-        if (OP == OP_GRAM || OP == OP_POLY) {
+        if (OP != OP_GRAM) {
+          float in[32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) unpack8(ecur[q], in + 8 * q);
           if (OP == OP_POLY) {
-            float a[32];
-            block_to_rows(stg, ecur, lane, a);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = fmaf(L.cc, x[c], L.cb * a[c]);
-          }
-          // Symmetric output: entry (r, c) with c >= r is owned by this tile;
-          // store it and mirror it to (c, r).  Chunks entirely below the
-          // diagonal of this warp's rows are skipped.
-          if (col0 + 31 < rbase) continue;
-          rows_to_stage(stg, x, lane);
-          stage_to_global(stg, P.out, P.ld_out, rbase, col0, M, N, lane, 0);
-          rows_to_stage_t(stg, x, lane);
-          // mirror block: rows col0.., columns rbase..; keep c' > r' there,
-          // i.e. (mirror row) > (mirror column)  <=>  column <= row - 1.
-          for (int k = 0; k < 4; ++k) {
-            const int r = (lane >> 2) + 8 * k;        // mirror row offset (a column of x)
-            const int c = (lane & 3) * 8;             // mirror column offset (a row of x)
-            const int grow = col0 + r, gcol = rbase + c;
-            if (grow >= N || gcol >= M) continue;
-            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * EPI_LD + c);
-            __nv_bfloat16* p = P.out + (long long)grow * P.ld_out + gcol;
-            if (gcol + 7 < grow && gcol + 8 <= M) {
-              *reinterpret_cast<uint4*>(p) = w;
-            } else {
-              const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                if (gcol + e < M && gcol + e < grow)
-                  p[e] = __ushort_as_bfloat16((uint16_t)((u[e >> 1] >> (16 * (e & 1))) & 0xFFFFu));
-            }
-          }
-          __syncwarp();
-        } else {
-          float a[32];
-          block_to_rows(stg, ecur, lane, a);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] = fmaf(L.ca, a[c], x[c]);
-          if (!FINAL) {
-            rows_to_stage(stg, x, lane);
-            stage_to_global(stg, P.out, P.ld_out, rbase, col0, M, N, lane, -1);
+            for (int c = 0; c < 32; ++c) x[c] = fmaf(L.cc, x[c], L.cb * in[c]);
           } else {
-            float xb[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) xb[c] = __bfloat162float(__float2bfloat16_rn(x[c]));
-            final_chunk(P, F, L.final_mode, stg, xb, rbase, col0, lane);
+            for (int c = 0; c < 32; ++c) x[c] = fmaf(L.ca, in[c], x[c]);
           }
+        }
+        if (OP == OP_GRAM || OP == OP_POLY) {
+          // Symmetric output.  rbase and col0 are multiples of 32, so this
+          // block lies above the diagonal (stored and mirrored), on it
+          // (symmetrised, stored once) or below it (owned by another tile).
+          if (col0 < rbase) continue;
+          if (lane == 0) bulk_wait_group_read<0>();    // both blocks free again
+          __syncwarp();
+          row_to_block(stg8, lane, x);
+          if (col0 == rbase) {
+            __syncwarp();
+            symmetrize_block(stg8, lane);
+          } else {
+            col_to_block(stg8 + EPI_BLOCK_BYTES, lane, x);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&P.tmOut, stg_s, col0, rbase);
+            if (col0 != rbase) tma_store_2d(&P.tmOut, stg_s + EPI_BLOCK_BYTES, rbase, col0);
+            bulk_commit_group();
+          }
+        } else if (!FINAL) {
+          uint8_t* blk = stg8 + (cc & 1) * EPI_BLOCK_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();    // the store from this block two chunks ago
+          __syncwarp();
+          row_to_block(blk, lane, x);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&P.tmOut, stg_s + (cc & 1) * EPI_BLOCK_BYTES, col0, rbase);
+            bulk_commit_group();
+          }
+        } else {
+          float xb[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) xb[c] = __bfloat162float(__float2bfloat16_rn(x[c]));
+          final_chunk(P, F, L.final_mode, stg, xb, rbase, col0, lane);
         }
       }
       tc_fence_before_sync();
@@ -505,6 +563,9 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         acc_phase ^= 1u;
       }
     }
+    // Stores must finish reading shared memory (and land) before the CTA exits.
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before_sync();
