@@ -11,15 +11,19 @@ Tolerances (from the arithmetic, stated per check):
   fp32 accumulation bound 2 K 2^-24 (|P||Q|)_ij of the product P Q (which
   matters only for entries that cancel to near zero), and differ on at most
   1% of entries.
-* orthogonalised update and new parameters: relative Frobenius error
-  <= 1e-2 over the step's update (all matrices of the call together), and
-  the new parameters per matrix.  The bf16 iteration is chaotic: directions
-  with small singular values are amplified up to a^5 ~ 485-fold, so the rare
-  accumulation-order roundings above grow with every iteration (0.01%, 0.05%,
-  0.25%, 0.5%, 0.8% after 1..5 iterations on GPT-2 shapes; the same algorithm
-  with a different fp32 summation order on the CPU moves X5 by 0.4%, and bf16
-  itself moves it 9% from the exact fp64 iteration).  Per matrix the update
-  is held to 1.5e-2 (largest observed: 1.005e-2, one 3072x768 matrix).
+* orthogonalised update (Delta p = -lr*s*X5) and new parameters: relative
+  Frobenius error <= 1e-2 for a single orthogonalisation and for a step from
+  zero momentum (measured <= 0.82%).  The bf16 iteration is chaotic:
+  directions with small singular values grow up to a = 3.44-fold per
+  iteration, so the rare accumulation-order roundings above grow with every
+  iteration (0.01%, 0.05%, 0.25%, 0.5%, 0.8% after 1..5 iterations).  The
+  tensor core accumulates in fp32 truncated toward zero; a CPU model of the
+  same algorithm with that accumulation (exact sums of 16 products, then an
+  fp32 accumulator truncated toward zero) lands as far from the oracle as
+  the GPU does (0.81% / 0.70% vs 0.78% / 0.66% at step 1, 0.99% / 0.87% vs
+  0.95% / 0.86% at step 2), while round-to-nearest fp32 would land at 0.4%.
+  Along a momentum trajectory the spectrum of u hardens and both reach
+  ~1.3% by step 8; those cases are held to X_TOL_TRAJ = 1.5e-2.
 """
 import math
 
@@ -37,8 +41,8 @@ from workloads import WORKLOADS, WorkloadStream, square_case
 pytestmark = pytest.mark.gpu
 
 COEFFS = (3.4445, -4.7750, 2.0315)
-X_TOL = 1e-2          # orthogonalised update of a step / one orthogonalisation
-X_TOL_MATRIX = 1.5e-2  # one matrix's update within a multi-matrix step
+X_TOL = 1e-2          # one orthogonalisation / a step from zero momentum
+X_TOL_TRAJ = 1.5e-2   # steps after momentum has accumulated (see module docstring)
 BUF_TOL = 1e-6
 
 
@@ -221,8 +225,8 @@ def _run_step(muon, params, grads, bufs, **kw):
 
 
 def _check_step(p_old, p_gpu, b_gpu, p_ref, b_ref, tol=X_TOL):
-    """Momentum buffers to 1e-6; new parameters to tol per matrix; the step's
-    update to tol over all matrices together and X_TOL_MATRIX per matrix."""
+    """Momentum buffers to 1e-6; new parameters and each matrix's update to
+    tol; the step's update over all matrices together to tol as well."""
     num = den = 0.0
     errs = []
     for po, pg, bg, pr, br in zip(p_old, p_gpu, b_gpu, p_ref, b_ref):
@@ -235,7 +239,7 @@ def _check_step(p_old, p_gpu, b_gpu, p_ref, b_ref, tol=X_TOL):
         num += float(np.sum((dp_g - dp_r) ** 2))
         den += float(np.sum(dp_r ** 2))
         errs.append((po.shape, rel_fro(dp_g, dp_r)))
-        assert errs[-1][1] <= max(tol, X_TOL_MATRIX), errs[-1]
+        assert errs[-1][1] <= tol, errs[-1]
     if den > 0:
         assert math.sqrt(num / den) <= tol, errs
 
@@ -293,7 +297,7 @@ def test_step_workloads_consecutive(muon, name, steps):
     b_d = [to_f32(b) for b in bufs]
     p_ref = [p.copy() for p in params]
     b_ref = [b.copy() for b in bufs]
-    for _ in range(steps):
+    for k in range(steps):
         grads = st.next_grads()
         p_old = [p.copy() for p in p_ref]
         muon.step(p_d, [to_f32(g) for g in grads], b_d, lr=wl.lr, beta=wl.beta,
@@ -301,7 +305,8 @@ def test_step_workloads_consecutive(muon, name, steps):
         torch.cuda.synchronize()
         p_ref, b_ref = muon_step_ref(p_ref, grads, b_ref, lr=wl.lr, beta=wl.beta,
                                      nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
-        _check_step(p_old, p_d, b_d, p_ref, b_ref)
+        zero_momentum = k == 0 and wl.buf_std == 0
+        _check_step(p_old, p_d, b_d, p_ref, b_ref, tol=X_TOL if zero_momentum else X_TOL_TRAJ)
         # keep the two trajectories on the same state, so that each step is
         # compared from identical inputs
         for i in range(len(p_d)):
@@ -324,8 +329,9 @@ def test_step_gpt2_124m_full_size_sampled(muon):
     p_ref, b_ref = muon_step_ref([params[i] for i in sample], [grads[i] for i in sample],
                                  [bufs[i] for i in sample], lr=wl.lr, beta=wl.beta,
                                  nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    # momentum is warm-started (N(0, 0.1^2)), so this is a trajectory step
     _check_step([params[i] for i in sample], [p_d[i] for i in sample], [b_d[i] for i in sample],
-                p_ref, b_ref)
+                p_ref, b_ref, tol=X_TOL_TRAJ)
     # property at full size: every momentum buffer matches the one-rounding form
     for i in range(0, 48, 7):
         br, _ = momentum_ref(grads[i], bufs[i], wl.beta, wl.nesterov)
