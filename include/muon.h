@@ -136,6 +136,38 @@ MUON_API int muon_xupdate(const uint16_t* b, int64_t ld_b, const uint16_t* x, in
                  uint16_t* x_out, int64_t ld_out, int64_t m, int64_t n, float ca,
                  void* stream);
 
+/*
+ * muon_momentum_normalize_noalloc -- the same computation as
+ * muon_momentum_normalize, for callers that cannot allocate device memory
+ * when they run the optimizer (a host whose device memory is all handed to
+ * its own pool allocator, or a process that must not grow its footprint
+ * after start-up).  It allocates nothing: its scratch (work queue, per-matrix
+ * counters and flags, norm partials) lives in a fixed array of about 200 KB
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits.  There is no counterpart of this entry point on
+ * the pages; it is an interface choice of this library.
+ *
+ * Arguments as for muon_momentum_normalize, plus:
+ *   dev_status  device pointer to one int owned by the caller (or NULL).  A
+ *               device-side wait that runs out stores MUON_ERR_TIMEOUT there
+ *               (the first error wins; the caller zeroes it).  With NULL such
+ *               a failure is not reported.  muon_status() does not see it.
+ * Limits: at most MUON_NOALLOC_MAX_MATRICES matrices, and at most
+ * MUON_NOALLOC_MAX_ITEMS work items, where a matrix of r x c elements takes
+ * 2 * ceil(ceil(r/64) * ceil(c/64) / 4) items (about 134M elements in all);
+ * larger calls return MUON_ERR_UNSUPPORTED before doing anything.
+ * The first call on a device takes the fixed array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array: calls whose
+ * executions overlap on the GPU race, so order them on one stream.
+ */
+#define MUON_NOALLOC_MAX_MATRICES 64
+#define MUON_NOALLOC_MAX_ITEMS 16384
+MUON_API int muon_momentum_normalize_noalloc(const float* const* grads, float* const* bufs,
+                                             uint16_t* const* x0, const int64_t* x0_ld,
+                                             const int64_t* shapes, int n, float beta,
+                                             int nesterov, int* dev_status, void* stream);
+
 /* muon_status -- synchronises the stream, then returns (and clears) the
  * device-side status of the current device: MUON_OK or MUON_ERR_TIMEOUT;
  * MUON_ERR_CUDA if the synchronisation itself failed. */

@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so"
 EXPORTS = ("muon_step", "muon_orthogonalize", "muon_momentum_normalize", "muon_gram", "muon_poly",
            "muon_xupdate", "muon_status", "muon_error_string", "muon_set_wait_limit_ns",
            "muon_workspace_bytes", "muon_release", "muon_version", "muon_profile_begin",
-           "muon_profile_end")
+           "muon_profile_end", "muon_momentum_normalize_noalloc")
 
 PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply")
 
@@ -76,6 +76,7 @@ def library() -> ctypes.CDLL:
         "muon_version": (ctypes.c_char_p, []),
         "muon_profile_begin": (None, []),
         "muon_profile_end": (i, [ctypes.POINTER(ctypes.c_double), _I64P, i]),
+        "muon_momentum_normalize_noalloc": (i, [_PP, _PP, _PP, _I64P, _I64P, i, f, i, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -270,3 +271,22 @@ def profile_end() -> dict:
     if code < 0:
         raise MuonError(code, "muon_profile_end")
     return {PROFILE_KINDS[i]: (float(ms[i]), int(n[i])) for i in range(k)}
+
+
+def momentum_normalize_noalloc(grads, bufs, x0s, beta=0.95, nesterov=True, dev_status=None,
+                               stream=None) -> int:
+    """The fused first kernel through the allocation-free entry point.
+
+    For callers that must not allocate device memory while stepping: the
+    library's scratch is a fixed array compiled into it.  ``x0s`` are
+    caller-allocated bf16 buffers (min(r,c) x ld, ld % 8 == 0, ld >= max(r,c));
+    ``dev_status`` an optional int32 CUDA tensor of one element that receives
+    a device-side timeout.  Returns the status code (0 on success).
+    """
+    n = len(grads)
+    shapes = [v for g in grads for v in g.shape]
+    lds = [x.shape[1] for x in x0s]
+    return library().muon_momentum_normalize_noalloc(
+        _ptr_array(grads), _ptr_array(bufs), _ptr_array(x0s), (ctypes.c_int64 * max(n, 1))(*lds),
+        (ctypes.c_int64 * max(len(shapes), 1))(*shapes), n, float(beta), int(bool(nesterov)),
+        None if dev_status is None else dev_status.data_ptr(), _stream_ptr(stream))
