@@ -126,7 +126,7 @@ def source_hash():
 def recorded_traffic(kind):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "dram_traffic_gpt2_124m.txt")
     try:
         with open(path) as f:
             d = json.load(f)
