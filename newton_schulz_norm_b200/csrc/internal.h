@@ -30,9 +30,19 @@ constexpr int EPI_LD = 40;                  // padded staging pitch (bf16) of th
 constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;       // one 32 x 32 bf16 block, 64-byte swizzled
 constexpr int EPI_STAGE_BYTES = 2 * EPI_BLOCK_BYTES;   // two blocks per epilogue warp
 constexpr int OUT_BOX = 32;                 // TMA store box: 32 x 32 bf16, 64-byte swizzle
-constexpr int GEMM_BAR_BYTES = 256;
+constexpr int GEMM_BAR_BYTES = 512;
 constexpr size_t GEMM_SMEM_BYTES =
     size_t(STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
+
+// The last X update is bound by the fp32 parameter read-modify-write, not by
+// the tensor cores, so it trades main-loop stages for a per-warp ring of
+// parameter blocks moved by TMA (32 x 32 fp32, 128-byte swizzle).
+constexpr int FINAL_STAGES = 2;
+constexpr int P_RING = 4;                    // parameter blocks per epilogue warp
+constexpr int P_BLOCK_BYTES = 32 * 32 * 4;
+constexpr int FINAL_EPI_BYTES = P_RING * P_BLOCK_BYTES;   // per epilogue warp
+constexpr size_t FINAL_SMEM_BYTES =
+    size_t(FINAL_STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * FINAL_EPI_BYTES + 1024 + GEMM_BAR_BYTES;
 
 enum NsOp : int { OP_GRAM = 0, OP_POLY = 1, OP_UPDATE = 2 };
 
@@ -78,6 +88,10 @@ struct NsLaunch {
   const NsTile* tiles;
   int ntiles;
   int final_mode;
+  // Final FINAL_PARAM launch only: one tensor map per matrix (indexed by
+  // NsProblem::slot) over the stored fp32 parameters, 32 x 32 boxes with
+  // 128-byte swizzle; nullptr selects the register read-modify-write path.
+  const CUtensorMap* pmaps;
   float ca, cb, cc;
   unsigned long long limit_ns;
   int* status;

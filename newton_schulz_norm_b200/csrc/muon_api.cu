@@ -85,6 +85,21 @@ bool make_out_map(CUtensorMap* map, const void* base, long long rows, long long 
   return r == CUDA_SUCCESS;
 }
 
+// fp32 parameter map for the last X update: 32 x 32 boxes, 128-byte swizzle.
+// Needs the row pitch (cols * 4 bytes) to be a multiple of 16 bytes.
+bool make_param_map(CUtensorMap* map, const void* base, long long rows, long long cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 4)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- device memory arena
 
 struct Arena {
@@ -137,6 +152,10 @@ struct Plan {
   __nv_bfloat16* B = nullptr;
   NsPhase gram[2], poly, upd[2];
   K1Plan k1;
+  // Parameter tensor maps of the last X update, valid for the parameter
+  // pointers in pmap_for (rebuilt when a call passes other pointers).
+  DevBlock pmap_mem;
+  std::vector<const void*> pmap_for;
 };
 
 struct DeviceCtx {
@@ -554,10 +573,12 @@ int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, in
   return cuda_err(launch_k1(L, k1_grid(ctx, L.nitems), stream));
 }
 
-// The Newton-Schulz chain; the last update writes `final_mode` through F.
+// The Newton-Schulz chain; the last update writes `final_mode` through F
+// (through the parameter tensor maps `pmaps` when given).
 int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mode,
-           const FinalTable* F, cudaStream_t stream) {
+           const FinalTable* F, cudaStream_t stream, const CUtensorMap* pmaps = nullptr) {
   NsLaunch L;
+  L.pmaps = nullptr;
   L.ca = co[0];
   L.cb = co[1];
   L.cc = co[2];
@@ -587,6 +608,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     L.tiles = P->upd[par].tiles;
     L.ntiles = P->upd[par].ntiles;
     L.final_mode = (s == ns_steps - 1) ? final_mode : FINAL_NONE;
+    L.pmaps = (s == ns_steps - 1) ? pmaps : nullptr;
     {
       ProfScope ps(L.final_mode == FINAL_NONE ? PK_UPDATE : PK_FINAL, stream);
       e = launch_ns_gemm(OP_UPDATE, L, F, std::min(L.ntiles, ctx->num_sms), stream);
@@ -622,6 +644,41 @@ std::vector<long long> shape_key(char kind, const std::vector<Geom>& geom) {
   return key;
 }
 
+// Tensor maps over the caller's parameters for the TMA path of the last X
+// update.  They depend on the pointers, so they are rebuilt (after the stream
+// has drained, since queued kernels may still read the old ones) whenever a
+// call passes other pointers than the previous one.  Shapes whose row pitch
+// is not a multiple of 16 bytes use the register path (*out = nullptr).
+int ensure_param_maps(Plan* P, float* const* params, int n, cudaStream_t stream,
+                      const CUtensorMap** out) {
+  *out = nullptr;
+  for (int i = 0; i < n; ++i)
+    if (P->geom[i].c % 4 != 0) return MUON_OK;
+  std::vector<const void*> want(params, params + n);
+  if (P->pmap_mem.ptr && P->pmap_for == want) {
+    *out = reinterpret_cast<const CUtensorMap*>(P->pmap_mem.ptr);
+    return MUON_OK;
+  }
+  if (!P->pmap_mem.ptr) {
+    if (cudaMalloc(&P->pmap_mem.ptr, sizeof(CUtensorMap) * n) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_NOMEM;
+    }
+    P->pmap_mem.bytes = sizeof(CUtensorMap) * n;
+  } else if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    return MUON_ERR_CUDA;
+  }
+  std::vector<CUtensorMap> maps(n);
+  for (int i = 0; i < n; ++i)
+    if (!make_param_map(&maps[i], params[i], P->geom[i].r, P->geom[i].c)) return MUON_ERR_CUDA;
+  if (cudaMemcpy(P->pmap_mem.ptr, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  P->pmap_for = want;
+  *out = reinterpret_cast<const CUtensorMap*>(P->pmap_mem.ptr);
+  return MUON_OK;
+}
+
 int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, float* const* bufs,
                const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
                const float* co, cudaStream_t stream) {
@@ -645,7 +702,10 @@ int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, 
     std::vector<void*> dst(params, params + n);
     return run_apply(P, FINAL_PARAM, dst.data(), F.scale, stream);
   }
-  return run_ns(ctx, P, ns_steps, co, FINAL_PARAM, &F, stream);
+  const CUtensorMap* pmaps = nullptr;
+  rc = ensure_param_maps(P, params, n, stream, &pmaps);
+  if (rc) return rc;
+  return run_ns(ctx, P, ns_steps, co, FINAL_PARAM, &F, stream, pmaps);
 }
 
 }  // namespace
@@ -811,6 +871,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
     ctx->stage_plans[key] = std::move(np);
   }
   NsLaunch L;
+  L.pmaps = nullptr;
   L.probs = P->poly.probs;
   L.tiles = P->poly.tiles;
   L.ntiles = P->poly.ntiles;

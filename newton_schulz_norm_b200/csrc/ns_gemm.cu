@@ -213,26 +213,64 @@ __device__ __forceinline__ void rows_to_stage_t(uint16_t* stg, const float (&x)[
   __syncwarp();
 }
 
-// The final iteration's output: X (bf16-rounded) applied to or written into
-// the caller's buffer, in the stored orientation.
-__device__ __forceinline__ void final_chunk(const NsProblem& P, const FinalTable* F, int mode,
+// The final iteration's output: X (bf16-rounded) applied to, or written
+// into, the caller's buffer in the stored orientation.  The parameter block a
+// lane needs is fetched by final_load one chunk ahead of final_apply, so the
+// fp32 read-modify-write of one chunk overlaps the reads of the next.
+//
+// Lane layout of the 32x32 block: transposed targets (X(row, col) at
+// [col][row]) use lane = row, value c = column (each column one coalesced
+// 128-byte segment); other targets use lane -> rows (lane>>3) + 4k,
+// columns (lane&7)*4 .. +3 (4 rows x 128 contiguous bytes per instruction).
+__device__ __forceinline__ void final_load(const NsProblem& P, const FinalTable* F, int mode,
+                                           int rbase, int col0, int lane, float (&pv)[32]) {
+  if (mode != FINAL_PARAM) return;
+  const int M = P.M, N = P.N;
+  const long long ldf = P.ld_final;
+  const float* base = reinterpret_cast<const float*>(F->ptr[P.slot]);
+  if (P.transposed) {
+    const int row = rbase + lane;
+    const bool rok = row < M;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      pv[c] = (rok && col0 + c < N) ? base[(long long)(col0 + c) * ldf + row] : 0.f;
+    return;
+  }
+  const bool vec_ok = (ldf & 3) == 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int grow = rbase + (lane >> 3) + 4 * k, gcol = col0 + (lane & 7) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (grow < M && gcol < N) {
+      const float* q = base + (long long)grow * ldf + gcol;
+      if (vec_ok && gcol + 4 <= N) {
+        v = *reinterpret_cast<const float4*>(q);
+      } else {
+        v.x = q[0];
+        if (gcol + 1 < N) v.y = q[1];
+        if (gcol + 2 < N) v.z = q[2];
+        if (gcol + 3 < N) v.w = q[3];
+      }
+    }
+    pv[4 * k + 0] = v.x;
+    pv[4 * k + 1] = v.y;
+    pv[4 * k + 2] = v.z;
+    pv[4 * k + 3] = v.w;
+  }
+}
+
+__device__ __forceinline__ void final_apply(const NsProblem& P, const FinalTable* F, int mode,
                                             uint16_t* stg, const float (&xb)[32], int rbase,
-                                            int col0, int lane) {
+                                            int col0, int lane, const float (&pv)[32]) {
   const int M = P.M, N = P.N;
   const int slot = P.slot;
   const long long ldf = P.ld_final;
   const float neg_scale = -F->scale[slot];
   if (P.transposed) {
-    // X(row, col) lands at [col][row]; lanes hold consecutive rows, so each
-    // column is one coalesced 128-byte segment.  Loads are issued together.
     const int row = rbase + lane;
     const bool rok = row < M;
     if (mode == FINAL_PARAM) {
       float* base = reinterpret_cast<float*>(F->ptr[slot]);
-      float pv[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        pv[c] = (rok && col0 + c < N) ? base[(long long)(col0 + c) * ldf + row] : 0.f;
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (rok && col0 + c < N) base[(long long)(col0 + c) * ldf + row] = fmaf(neg_scale, xb[c], pv[c]);
@@ -255,84 +293,64 @@ __device__ __forceinline__ void final_chunk(const NsProblem& P, const FinalTable
                     lane, -1);
     return;
   }
-  // fp32 target, coalesced: lane handles row (lane>>3) + 4k, columns
-  // (lane&7)*4 .. +3 (each instruction covers 4 rows x 128 contiguous bytes).
   float* base = reinterpret_cast<float*>(F->ptr[slot]);
   const bool vec_ok = (ldf & 3) == 0;
-  float4 pv[8];
-  if (mode == FINAL_PARAM) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int grow = rbase + (lane >> 3) + 4 * k, gcol = col0 + (lane & 7) * 4;
-      pv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (grow < M && gcol < N) {
-        const float* p = base + (long long)grow * ldf + gcol;
-        if (vec_ok && gcol + 4 <= N) {
-          pv[k] = *reinterpret_cast<const float4*>(p);
-        } else {
-          pv[k].x = p[0];
-          if (gcol + 1 < N) pv[k].y = p[1];
-          if (gcol + 2 < N) pv[k].z = p[2];
-          if (gcol + 3 < N) pv[k].w = p[3];
-        }
-      }
-    }
-  }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const int r = (lane >> 3) + 4 * k, c = (lane & 7) * 4;
     const int grow = rbase + r, gcol = col0 + c;
     if (grow >= M || gcol >= N) continue;
     const uint2 w = *reinterpret_cast<const uint2*>(stg + r * EPI_LD + c);
-    float x4[4] = {bf16_bits_to_float(w.x & 0xFFFFu), bf16_bits_to_float(w.x >> 16),
-                   bf16_bits_to_float(w.y & 0xFFFFu), bf16_bits_to_float(w.y >> 16)};
+    const float x4[4] = {bf16_bits_to_float(w.x & 0xFFFFu), bf16_bits_to_float(w.x >> 16),
+                         bf16_bits_to_float(w.y & 0xFFFFu), bf16_bits_to_float(w.y >> 16)};
     float4 o;
     if (mode == FINAL_PARAM) {
-      o.x = fmaf(neg_scale, x4[0], pv[k].x);
-      o.y = fmaf(neg_scale, x4[1], pv[k].y);
-      o.z = fmaf(neg_scale, x4[2], pv[k].z);
-      o.w = fmaf(neg_scale, x4[3], pv[k].w);
+      o.x = fmaf(neg_scale, x4[0], pv[4 * k + 0]);
+      o.y = fmaf(neg_scale, x4[1], pv[4 * k + 1]);
+      o.z = fmaf(neg_scale, x4[2], pv[4 * k + 2]);
+      o.w = fmaf(neg_scale, x4[3], pv[4 * k + 3]);
     } else {
       o = make_float4(x4[0], x4[1], x4[2], x4[3]);
     }
-    float* p = base + (long long)grow * ldf + gcol;
+    float* q = base + (long long)grow * ldf + gcol;
     if (vec_ok && gcol + 4 <= N) {
-      *reinterpret_cast<float4*>(p) = o;
+      *reinterpret_cast<float4*>(q) = o;
     } else {
-      p[0] = o.x;
-      if (gcol + 1 < N) p[1] = o.y;
-      if (gcol + 2 < N) p[2] = o.z;
-      if (gcol + 3 < N) p[3] = o.w;
+      q[0] = o.x;
+      if (gcol + 1 < N) q[1] = o.y;
+      if (gcol + 2 < N) q[2] = o.z;
+      if (gcol + 3 < N) q[3] = o.w;
     }
   }
   __syncwarp();
 }
 
-// FINAL = the last X update (writes through FinalTable instead of the next
-// iterate); it fetches its epilogue input per chunk to leave registers for
-// the fp32 read-modify-write of the parameters.
 template <int OP, bool FINAL>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
+  constexpr int NST = FINAL ? FINAL_STAGES : STAGES;            // main-loop ring depth
+  constexpr int EPI_REGION = FINAL ? FINAL_EPI_BYTES : EPI_STAGE_BYTES;   // per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;     // 128B-swizzle atoms need 1 KB alignment
   uint8_t* gbase = smem_raw + (sbase - raw);
-  uint16_t* epi_stage = reinterpret_cast<uint16_t*>(gbase + STAGES * STAGE_BYTES);
-  const uint32_t bar0 = sbase + STAGES * STAGE_BYTES + EPI_WARPS * EPI_STAGE_BYTES;
-  // barrier layout: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  const uint32_t bar0 = sbase + NST * STAGE_BYTES + EPI_WARPS * EPI_REGION;
+  // barrier layout: full[NST], empty[NST], tfull[2], tempty[2], drain,
+  // then (final kernel) P_RING parameter-block barriers per epilogue warp
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES +
-                                                    EPI_WARPS * EPI_STAGE_BYTES + 8 * (2 * STAGES + 5));
+  auto empty_bar = [&](int s) { return bar0 + 8u * (NST + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * NST + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * NST + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * NST + 4);
+  const uint32_t pbar_base = bar0 + 8u * (2 * NST + 5);
+  constexpr int NBARS = 2 * NST + 5 + (FINAL ? EPI_WARPS * P_RING : 0);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + NST * STAGE_BYTES +
+                                                    EPI_WARPS * EPI_REGION + 8 * NBARS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
@@ -341,6 +359,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       mbar_init(tempty_bar(a), EPI_THREADS);
     }
     mbar_init(drain_bar, 1);
+    if (FINAL)
+      for (int b = 0; b < EPI_WARPS * P_RING; ++b) mbar_init(pbar_base + 8u * b, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -391,7 +411,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             for (int q = 0; q < BN / BOX; ++q)
               tma_load_2d(sB + q * BOX_BYTES, &P->tmB, fb, k0, tile.j0 + q * BOX);
           }
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -399,7 +419,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       }
       // Never leave with copies in flight: wait (bounded) for the last load
       // armed on each stage.  On the normal path these have all landed.
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < NST; ++s)
         if (armed_mask & (1u << s))
           if (!mbar_wait(full_bar(s), (armed_parity >> s) & 1u, kDrainLimitNs))
             record_status(L.status, MUON_ERR_TIMEOUT);
@@ -446,7 +466,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             umma_f16(d_tmem, adesc, bdesc, idesc, (kc | kk) != 0 ? 1u : 0u);
           }
           umma_commit(empty_bar(stage));
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -467,9 +487,142 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     const int ew = warp - 2;                    // 0..7
     const int quarter = warp & 3;               // TMEM lanes this warp may access
     const int half = ew >> 2;                   // which 4 of the 8 column chunks
-    uint8_t* stg8 = gbase + STAGES * STAGE_BYTES + ew * EPI_STAGE_BYTES;
+    uint8_t* stg8 = gbase + NST * STAGE_BYTES + ew * EPI_REGION;
     uint16_t* stg = reinterpret_cast<uint16_t*>(stg8);
     const uint32_t stg_s = smem_addr(stg8);
+    if (FINAL && L.pmaps != nullptr && L.final_mode == FINAL_PARAM) {
+      // ---- last iteration, parameter blocks through a per-warp TMA ring.
+      // Chunk h of this warp (4 per tile, tiles in the CTA's round-robin
+      // order) owns ring slot h % P_RING.  The block for chunk h + 2 is loaded
+      // while chunk h is combined; a slot is reloaded only after the store
+      // that last used it has finished reading shared memory.
+      uint8_t* ring = stg8;
+      const uint32_t ring_s = smem_addr(ring);
+      const uint32_t pbar0 = pbar_base + 8u * (ew * P_RING);
+      const int ntl = ((int)blockIdx.x < L.ntiles) ? (L.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      const int nch = ntl * CHUNKS_PER_WARP;
+      uint32_t pphase = 0;    // per slot: parity of its next completion
+      uint32_t pending = 0;   // per slot: a load is in flight and not yet consumed
+      auto chunk_info = [&](int h, const NsProblem*& Pp, int& rb, int& c0) -> bool {
+        const NsTile tl = L.tiles[blockIdx.x + (h / CHUNKS_PER_WARP) * gridDim.x];
+        Pp = L.probs + tl.prob;
+        rb = tl.i0 + quarter * 32;
+        c0 = tl.j0 + half * (CHUNKS_PER_WARP * 32) + (h % CHUNKS_PER_WARP) * 32;
+        return rb < Pp->M && c0 < Pp->N;
+      };
+      auto issue = [&](int h) {          // every lane tracks the state; lane 0 issues
+        if (h >= nch) return;
+        const NsProblem* Pp;
+        int rb, c0;
+        if (!chunk_info(h, Pp, rb, c0)) return;
+        const int b = h % P_RING;
+        if (lane == 0) {
+          const uint32_t bar = pbar0 + 8u * b;
+          mbar_arrive_expect_tx(bar, P_BLOCK_BYTES);
+          const CUtensorMap* pm = L.pmaps + Pp->slot;
+          // transposed targets: X(i, j) is p[j][i], so the block starts at p(col0, rbase)
+          if (Pp->transposed) tma_load_2d(ring_s + b * P_BLOCK_BYTES, pm, bar, rb, c0);
+          else tma_load_2d(ring_s + b * P_BLOCK_BYTES, pm, bar, c0, rb);
+        }
+        pending |= 1u << b;
+      };
+      issue(0);
+      issue(1);
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint4 ecur[4], enext[4];
+      for (int h = 0; h < nch; ++h) {
+        const int cc = h % CHUNKS_PER_WARP;
+        const NsProblem* Pp;
+        int rb, col0;
+        const bool live = chunk_info(h, Pp, rb, col0);
+        const NsProblem& P = *Pp;
+        const int row = rb + lane;
+        if (cc == 0) {
+          load_row(P.epi, P.ld_epi, row, col0, P.M, P.N, ecur);
+          if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
+            record_status(L.status, MUON_ERR_TIMEOUT);
+            break;
+          }
+          tc_fence_after_sync();
+        }
+        if (lane == 0) bulk_wait_group_read<1>();   // the store of chunk h - 2 has read its slot
+        __syncwarp();
+        issue(h + 2);
+        if (cc + 1 < CHUNKS_PER_WARP) load_row(P.epi, P.ld_epi, row, col0 + 32, P.M, P.N, enext);
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
+                               half * (CHUNKS_PER_WARP * 32) + cc * 32, v);
+        tmem_ld_wait();
+        bool stop = false;
+        if (live) {
+          const int b = h % P_RING;
+          const bool got = mbar_wait(pbar0 + 8u * b, (pphase >> b) & 1u, limit);
+          pphase ^= 1u << b;
+          pending &= ~(1u << b);
+          if (!got) {
+            record_status(L.status, MUON_ERR_TIMEOUT);
+            stop = true;
+          } else {
+            float in[32], xb[32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) unpack8(ecur[q], in + 8 * q);
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              xb[c] = __bfloat162float(__float2bfloat16_rn(fmaf(L.ca, in[c], __uint_as_float(v[c]))));
+            const float neg_scale = -F->scale[P.slot];
+            uint8_t* blk = ring + b * P_BLOCK_BYTES;
+            // 32 x 32 fp32 block, 128-byte swizzle: element (r, c) at
+            // r*128 + (((c >> 2) ^ (r & 7)) << 4) + (c & 3)*4
+            if (P.transposed) {
+              // this lane's X row is block column `lane`; X column c is block row c
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                float* q = reinterpret_cast<float*>(blk + c * 128 + ((((lane >> 2) ^ (c & 7))) << 4) +
+                                                    ((lane & 3) << 2));
+                *q = fmaf(neg_scale, xb[c], *q);
+              }
+            } else {
+#pragma unroll
+              for (int qd = 0; qd < 8; ++qd) {
+                float4* q = reinterpret_cast<float4*>(blk + lane * 128 + ((qd ^ (lane & 7)) << 4));
+                float4 pv = *q;
+                pv.x = fmaf(neg_scale, xb[4 * qd + 0], pv.x);
+                pv.y = fmaf(neg_scale, xb[4 * qd + 1], pv.y);
+                pv.z = fmaf(neg_scale, xb[4 * qd + 2], pv.z);
+                pv.w = fmaf(neg_scale, xb[4 * qd + 3], pv.w);
+                *q = pv;
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const CUtensorMap* pm = L.pmaps + P.slot;
+              if (P.transposed) tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, rb, col0);
+              else tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, col0, rb);
+            }
+          }
+        }
+        if (lane == 0) bulk_commit_group();        // one group per chunk, empty or not
+        if (stop) break;
+        if (cc + 1 < CHUNKS_PER_WARP) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) ecur[q] = enext[q];
+        } else {
+          tc_fence_before_sync();
+          mbar_arrive(tempty_bar(acc));
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      // Loads issued but never consumed (only after a timeout) land before exit.
+      for (int b = 0; b < P_RING; ++b)
+        if (pending & (1u << b))
+          if (!mbar_wait(pbar0 + 8u * b, (pphase >> b) & 1u, kDrainLimitNs))
+            record_status(L.status, MUON_ERR_TIMEOUT);
+    } else {
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
@@ -484,6 +637,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       uint4 ein[NPRE > 0 ? NPRE : 1][4];
 #pragma unroll
       for (int cc = 0; cc < NPRE; ++cc) load_row(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
+      float pcur[32];
+      if (FINAL) final_load(P, F, L.final_mode, rbase, cbase, lane, pcur);
       if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
         record_status(L.status, MUON_ERR_TIMEOUT);
         break;
@@ -492,12 +647,41 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
                              half * (CHUNKS_PER_WARP * 32);
       const bool rows_live = rbase < M;
-      constexpr int UNROLL = FINAL ? 1 : CHUNKS_PER_WARP;
-#pragma unroll UNROLL
+      if (FINAL) {
+        // Last iteration: one chunk of input and parameters in flight ahead.
+#pragma unroll 1
+        for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
+          const int col0 = cbase + cc * 32;
+          uint4 enext[4];
+          float pnext[32];
+          if (cc + 1 < CHUNKS_PER_WARP) {
+            load_row(P.epi, P.ld_epi, row, col0 + 32, M, N, enext);
+            final_load(P, F, L.final_mode, rbase, col0 + 32, lane, pnext);
+          }
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + cc * 32, v);
+          tmem_ld_wait();
+          if (rows_live && col0 < N) {                // warp-uniform
+            float in[32], xb[32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) unpack8(ein[0][q], in + 8 * q);
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              xb[c] = __bfloat162float(__float2bfloat16_rn(fmaf(L.ca, in[c], __uint_as_float(v[c]))));
+            final_apply(P, F, L.final_mode, stg, xb, rbase, col0, lane, pcur);
+          }
+          if (cc + 1 < CHUNKS_PER_WARP) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ein[0][q] = enext[q];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pcur[c] = pnext[c];
+          }
+        }
+      } else {
+#pragma unroll
       for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
         const int col0 = cbase + cc * 32;
-        uint4 (&ecur)[4] = ein[FINAL ? 0 : (NPRE > 0 ? cc : 0)];
-        if (FINAL && cc > 0) load_row(P.epi, P.ld_epi, row, col0, M, N, ecur);
+        uint4 (&ecur)[4] = ein[NPRE > 0 ? cc : 0];
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_ld_wait();
@@ -538,7 +722,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             if (col0 != rbase) tma_store_2d(&P.tmOut, stg_s + EPI_BLOCK_BYTES, rbase, col0);
             bulk_commit_group();
           }
-        } else if (!FINAL) {
+        } else {
           uint8_t* blk = stg8 + (cc & 1) * EPI_BLOCK_BYTES;
           if (lane == 0) bulk_wait_group_read<1>();    // the store from this block two chunks ago
           __syncwarp();
@@ -549,12 +733,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             tma_store_2d(&P.tmOut, stg_s + (cc & 1) * EPI_BLOCK_BYTES, col0, rbase);
             bulk_commit_group();
           }
-        } else {
-          float xb[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) xb[c] = __bfloat162float(__float2bfloat16_rn(x[c]));
-          final_chunk(P, F, L.final_mode, stg, xb, rbase, col0, lane);
         }
+      }
       }
       tc_fence_before_sync();
       mbar_arrive(tempty_bar(acc));
@@ -562,6 +742,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
     }
     // Stores must finish reading shared memory (and land) before the CTA exits.
     if (lane == 0) bulk_wait_group_all();
@@ -601,7 +782,7 @@ cudaError_t ns_gemm_setup(int /*device*/) {
                            (int)GEMM_SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)GEMM_SMEM_BYTES);
+                              (int)FINAL_SMEM_BYTES);
 }
 
 cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
@@ -615,7 +796,7 @@ cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int g
   } else if (L.final_mode == FINAL_NONE) {
     ns_gemm_kernel<OP_UPDATE><<<g, b, GEMM_SMEM_BYTES, stream>>>(L);
   } else {
-    ns_gemm_final_kernel<<<g, b, GEMM_SMEM_BYTES, stream>>>(L, *F);
+    ns_gemm_final_kernel<<<g, b, FINAL_SMEM_BYTES, stream>>>(L, *F);
   }
   return cudaGetLastError();
 }
