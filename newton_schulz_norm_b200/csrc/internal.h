@@ -11,16 +11,20 @@
 namespace muon {
 
 // ---------------------------------------------------------------- NS GEMM tiling
-// One CTA computes a BM x BN output tile with tcgen05.mma M=128, N=256, K=16,
-// fed by TMA through a STAGES-deep ring of BK-wide K slices.
-constexpr int BM = 128;
+// A CTA pair (cluster of 2, tcgen05 cta_group::2) computes a TILE_M x BN
+// output tile with M=256, N=256, K=16 MMAs issued by the pair's leader:
+// CTA r holds output rows [128 r, 128 r + 128) in its TMEM, A rows
+// [128 r, 128 r + 128) and B columns [128 r, 128 r + 128) in its shared
+// memory.  Each CTA streams BK-wide K slices through a STAGES-deep ring.
+constexpr int BM = 128;                     // output rows per CTA
+constexpr int TILE_M = 256;                 // output rows per CTA pair
 constexpr int BN = 256;
 constexpr int BK = 64;                      // one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int BOX = 64;                     // TMA box: 64 x 64 bf16 = 8 KB
 constexpr int BOX_BYTES = BOX * BOX * 2;
-constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
+constexpr int A_STAGE_BYTES = BM * BK * 2;          // 16 KB: this CTA's rows of A
+constexpr int B_STAGE_BYTES = (BN / 2) * BK * 2;    // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int EPI_WARPS = 8;                // two warps per TMEM lane quarter
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
@@ -37,7 +41,7 @@ constexpr size_t GEMM_SMEM_BYTES =
 // The last X update is bound by the fp32 parameter read-modify-write, not by
 // the tensor cores, so it trades main-loop stages for a per-warp ring of
 // parameter blocks moved by TMA (32 x 32 fp32, 128-byte swizzle).
-constexpr int FINAL_STAGES = 2;
+constexpr int FINAL_STAGES = 3;
 constexpr int P_RING = 4;                    // parameter blocks per epilogue warp
 constexpr int P_BLOCK_BYTES = 32 * 32 * 4;
 constexpr int FINAL_EPI_BYTES = P_RING * P_BLOCK_BYTES;   // per epilogue warp
@@ -161,6 +165,7 @@ struct ApplyLaunch {
 cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
                            cudaStream_t stream);
 cudaError_t ns_gemm_setup(int device);
+int ns_gemm_max_pairs();
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);
 int k1_blocks_per_sm();
 cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream);

@@ -162,6 +162,7 @@ struct DeviceCtx {
   int device = -1;
   int num_sms = 0;
   int k1_blocks_per_sm = 1;
+  int max_pairs = 1;           // co-resident CTA pairs of the GEMM kernels
   int* status = nullptr;
   std::map<std::vector<long long>, std::unique_ptr<Plan>> plans;
   std::map<std::vector<long long>, std::unique_ptr<Plan>> stage_plans;
@@ -235,6 +236,8 @@ int get_ctx(DeviceCtx** out) {
   if (cudaMalloc(&ctx->status, sizeof(int)) != cudaSuccess) return MUON_ERR_NOMEM;
   if (cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return MUON_ERR_CUDA;
   if (ns_gemm_setup(dev) != cudaSuccess) return MUON_ERR_CUDA;
+  ctx->max_pairs = ns_gemm_max_pairs();
+  if (ctx->max_pairs < 1) ctx->max_pairs = std::max(1, prop.multiProcessorCount / 2);
   ctx->k1_blocks_per_sm = k1_blocks_per_sm();   // persistent: as many CTAs as fit
   *out = ctx.get();
   g_ctx[dev] = std::move(ctx);
@@ -250,15 +253,16 @@ unsigned long long limit_ns() {
   return g_limit_ns;
 }
 
-// Gram / poly tiles: only tiles holding some entry on or above the diagonal.
+// Gram / poly tiles (TILE_M x BN, one per CTA pair): only tiles holding some
+// entry on or above the diagonal.
 void sym_tiles(std::vector<NsTile>& t, int prob, long long m, int kc) {
-  for (long long i0 = 0; i0 < m; i0 += BM)
+  for (long long i0 = 0; i0 < m; i0 += TILE_M)
     for (long long j0 = 0; j0 < m; j0 += BN)
       if (std::min(j0 + BN - 1, m - 1) >= i0) t.push_back({prob, (int)i0, (int)j0, kc});
 }
 
 void full_tiles(std::vector<NsTile>& t, int prob, long long m, long long n, int kc) {
-  for (long long i0 = 0; i0 < m; i0 += BM)
+  for (long long i0 = 0; i0 < m; i0 += TILE_M)
     for (long long j0 = 0; j0 < n; j0 += BN) t.push_back({prob, (int)i0, (int)j0, kc});
 }
 
@@ -545,6 +549,9 @@ int get_plan(DeviceCtx* ctx, std::vector<long long> key, const std::vector<Geom>
   return MUON_OK;
 }
 
+// Persistent GEMM grid: two CTAs (one cluster) per tile, at most one per SM.
+int pair_grid(DeviceCtx* ctx, int ntiles) { return 2 * std::max(1, std::min(ntiles, ctx->max_pairs)); }
+
 int k1_grid(DeviceCtx* ctx, int nitems) {
   return std::max(1, std::min(nitems, ctx->num_sms * ctx->k1_blocks_per_sm));
 }
@@ -593,7 +600,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     cudaError_t e;
     {
       ProfScope ps(PK_GRAM, stream);
-      e = launch_ns_gemm(OP_GRAM, L, nullptr, std::min(L.ntiles, ctx->num_sms), stream);
+      e = launch_ns_gemm(OP_GRAM, L, nullptr, pair_grid(ctx, L.ntiles), stream);
     }
     if (e != cudaSuccess) return MUON_ERR_CUDA;
     L.probs = P->poly.probs;
@@ -601,7 +608,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     L.ntiles = P->poly.ntiles;
     {
       ProfScope ps(PK_POLY, stream);
-      e = launch_ns_gemm(OP_POLY, L, nullptr, std::min(L.ntiles, ctx->num_sms), stream);
+      e = launch_ns_gemm(OP_POLY, L, nullptr, pair_grid(ctx, L.ntiles), stream);
     }
     if (e != cudaSuccess) return MUON_ERR_CUDA;
     L.probs = P->upd[par].probs;
@@ -611,7 +618,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     L.pmaps = (s == ns_steps - 1) ? pmaps : nullptr;
     {
       ProfScope ps(L.final_mode == FINAL_NONE ? PK_UPDATE : PK_FINAL, stream);
-      e = launch_ns_gemm(OP_UPDATE, L, F, std::min(L.ntiles, ctx->num_sms), stream);
+      e = launch_ns_gemm(OP_UPDATE, L, F, pair_grid(ctx, L.ntiles), stream);
     }
     if (e != cudaSuccess) return MUON_ERR_CUDA;
   }
@@ -881,7 +888,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
   L.cc = cc;
   L.limit_ns = limit_ns();
   L.status = ctx->status;
-  return cuda_err(launch_ns_gemm(op, L, nullptr, std::min(L.ntiles, ctx->num_sms),
+  return cuda_err(launch_ns_gemm(op, L, nullptr, pair_grid(ctx, L.ntiles),
                                  static_cast<cudaStream_t>(stream)));
 }
 

@@ -39,8 +39,8 @@ namespace {
 // shared memory or TMEM.
 constexpr unsigned long long kDrainLimitNs = 1000000000ull;
 
-constexpr uint32_t kIdescK = idesc_bf16_f32(BM, BN, 0);   // B operand K-major
-constexpr uint32_t kIdescMN = idesc_bf16_f32(BM, BN, 1);  // B operand MN-major
+constexpr uint32_t kIdescK = idesc_bf16_f32(TILE_M, BN, 0);   // pair MMA, B K-major
+constexpr uint32_t kIdescMN = idesc_bf16_f32(TILE_M, BN, 1);  // pair MMA, B MN-major
 constexpr int CHUNKS_PER_WARP = BN / 32 / 2;               // 4
 
 __device__ __forceinline__ void record_status(int* status, int code) {
@@ -348,15 +348,22 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pair: rank 0 (the leader) issues every MMA of the pair and owns the
+  // barriers the MMA waits on; both CTAs load their own operand halves and
+  // run their own epilogue on their own TMEM rows.
+  const uint32_t rank = cluster_cta_rank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1);
+  const int npairs = (int)(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);        // leader: its producer arms; both CTAs' bytes land
+      mbar_init(empty_bar(s), 1);       // both: the leader's MMA commit (multicast)
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), EPI_THREADS);
+      mbar_init(tfull_bar(a), 1);                    // both: leader's commit (multicast)
+      mbar_init(tempty_bar(a), 2 * EPI_THREADS);     // leader: both CTAs' epilogues
     }
     mbar_init(drain_bar, 1);
     if (FINAL)
@@ -365,51 +372,58 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  cluster_sync_all();            // both CTAs: barriers initialised, TMEM allocated
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const unsigned long long limit = L.limit_ns;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed_mask = 0, armed_parity = 0;
+      uint32_t armed_mask = 0, armed_parity = 0;   // leader: stages it armed
+      uint32_t used_mask = 0, used_parity = 0;     // stages this CTA loaded into
       bool ok = true;
-      for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+      for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
         const NsProblem* P = L.probs + tile.prob;
+        const int arow = tile.i0 + (int)rank * BM;           // this CTA's rows of A
+        const int bcol = tile.j0 + (int)rank * (BN / 2);     // this CTA's half of B
         for (int kc = 0; kc < tile.kc; ++kc) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit)) {
             record_status(L.status, MUON_ERR_TIMEOUT);
             ok = false;
             break;
           }
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          armed_mask |= 1u << stage;
-          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (leader) {
+            mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+            armed_mask |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          }
+          used_mask |= 1u << stage;
+          used_parity = (used_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = map_to_cta(full_bar(stage), 0);   // the leader's barrier
           const uint32_t sA = sbase + stage * STAGE_BYTES;
           const uint32_t sB = sA + A_STAGE_BYTES;
           const int k0 = kc * BK;
 #pragma unroll
           for (int q = 0; q < BM / BOX; ++q)
-            tma_load_2d(sA + q * BOX_BYTES, &P->tmA, fb, k0, tile.i0 + q * BOX);
+            tma_load_2d_pair(sA + q * BOX_BYTES, &P->tmA, fb, k0, arow + q * BOX);
           if (OP == OP_UPDATE) {
-            // B operand = X[k0:k0+64, j0:j0+256], MN-major: boxes along columns.
+            // B operand = X[k0:k0+64, bcol:bcol+128], MN-major: boxes along columns.
 #pragma unroll
-            for (int q = 0; q < BN / BOX; ++q)
-              tma_load_2d(sB + q * BOX_BYTES, &P->tmB, fb, tile.j0 + q * BOX, k0);
+            for (int q = 0; q < (BN / 2) / BOX; ++q)
+              tma_load_2d_pair(sB + q * BOX_BYTES, &P->tmB, fb, bcol + q * BOX, k0);
           } else {
-            // B operand = rows j0..j0+256 of X (or A), K-major.
+            // B operand = rows bcol..bcol+128 of X (or A), K-major.
 #pragma unroll
-            for (int q = 0; q < BN / BOX; ++q)
-              tma_load_2d(sB + q * BOX_BYTES, &P->tmB, fb, k0, tile.j0 + q * BOX);
+            for (int q = 0; q < (BN / 2) / BOX; ++q)
+              tma_load_2d_pair(sB + q * BOX_BYTES, &P->tmB, fb, k0, bcol + q * BOX);
           }
           if (++stage == NST) {
             stage = 0;
@@ -417,23 +431,29 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           }
         }
       }
-      // Never leave with copies in flight: wait (bounded) for the last load
-      // armed on each stage.  On the normal path these have all landed.
-      for (int s = 0; s < NST; ++s)
-        if (armed_mask & (1u << s))
+      // Never leave with copies in flight.  The leader waits for the last
+      // phase it armed on each stage (both CTAs' bytes land there); the peer
+      // waits for the MMA commit that follows its last load of each stage.
+      // On the normal path all of these have completed already.
+      for (int s = 0; s < NST; ++s) {
+        if (leader && (armed_mask & (1u << s)))
           if (!mbar_wait(full_bar(s), (armed_parity >> s) & 1u, kDrainLimitNs))
             record_status(L.status, MUON_ERR_TIMEOUT);
+        if (!leader && (used_mask & (1u << s)))
+          if (!mbar_wait(empty_bar(s), (used_parity >> s) & 1u, kDrainLimitNs))
+            record_status(L.status, MUON_ERR_TIMEOUT);
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader only)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       const uint32_t idesc = (OP == OP_UPDATE) ? kIdescMN : kIdescK;
-      for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+      for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit)) {
           record_status(L.status, MUON_ERR_TIMEOUT);
@@ -463,23 +483,23 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             } else {
               bdesc = smem_desc_sw128(sB + kk * 32, 16, 1024);
             }
-            umma_f16(d_tmem, adesc, bdesc, idesc, (kc | kk) != 0 ? 1u : 0u);
+            umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kc | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(empty_bar(stage));
+          umma_commit_pair(empty_bar(stage), 0x3);   // both CTAs' slices free
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(tfull_bar(acc));
+        umma_commit_pair(tfull_bar(acc), 0x3);       // both CTAs' accumulators ready
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // Drain: every MMA issued above completes before TMEM is released.
-      umma_commit(drain_bar);
+      umma_commit_pair(drain_bar, 0x1);
       if (!mbar_wait(drain_bar, 0, kDrainLimitNs)) record_status(L.status, MUON_ERR_TIMEOUT);
     }
   } else {
@@ -499,14 +519,14 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       uint8_t* ring = stg8;
       const uint32_t ring_s = smem_addr(ring);
       const uint32_t pbar0 = pbar_base + 8u * (ew * P_RING);
-      const int ntl = ((int)blockIdx.x < L.ntiles) ? (L.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      const int ntl = (pair < L.ntiles) ? (L.ntiles - 1 - pair) / npairs + 1 : 0;
       const int nch = ntl * CHUNKS_PER_WARP;
       uint32_t pphase = 0;    // per slot: parity of its next completion
       uint32_t pending = 0;   // per slot: a load is in flight and not yet consumed
       auto chunk_info = [&](int h, const NsProblem*& Pp, int& rb, int& c0) -> bool {
-        const NsTile tl = L.tiles[blockIdx.x + (h / CHUNKS_PER_WARP) * gridDim.x];
+        const NsTile tl = L.tiles[pair + (h / CHUNKS_PER_WARP) * npairs];
         Pp = L.probs + tl.prob;
-        rb = tl.i0 + quarter * 32;
+        rb = tl.i0 + (int)rank * BM + quarter * 32;
         c0 = tl.j0 + half * (CHUNKS_PER_WARP * 32) + (h % CHUNKS_PER_WARP) * 32;
         return rb < Pp->M && c0 < Pp->N;
       };
@@ -610,7 +630,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           for (int q = 0; q < 4; ++q) ecur[q] = enext[q];
         } else {
           tc_fence_before_sync();
-          mbar_arrive(tempty_bar(acc));
+          mbar_arrive_remote(map_to_cta(tempty_bar(acc), 0));
           if (++acc == 2) {
             acc = 0;
             acc_phase ^= 1u;
@@ -625,11 +645,11 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     } else {
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
+    for (int t = pair; t < L.ntiles; t += npairs) {
       const NsTile tile = L.tiles[t];
       const NsProblem& P = L.probs[tile.prob];
       const int M = P.M, N = P.N;
-      const int rbase = tile.i0 + quarter * 32;
+      const int rbase = tile.i0 + (int)rank * BM + quarter * 32;
       const int row = rbase + lane;
       const int cbase = tile.j0 + half * (CHUNKS_PER_WARP * 32);
       // Epilogue input (this lane's row), fetched before the accumulator is ready.
@@ -737,7 +757,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       }
       }
       tc_fence_before_sync();
-      mbar_arrive(tempty_bar(acc));
+      mbar_arrive_remote(map_to_cta(tempty_bar(acc), 0));   // the leader's MMA waits on it
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -749,12 +769,14 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     __syncwarp();
   }
 
+  // Both CTAs finished: no MMA writes either TMEM and no arrival targets
+  // either CTA's barriers any more.
   tc_fence_before_sync();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -785,20 +807,48 @@ cudaError_t ns_gemm_setup(int /*device*/) {
                               (int)FINAL_SMEM_BYTES);
 }
 
+// How many CTA pairs (clusters of two) can be resident at once.
+int ns_gemm_max_pairs() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel<OP_UPDATE>, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Launched as clusters of two CTAs (the MMA pair); grid is even.
 cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
                            cudaStream_t stream) {
   if (L.ntiles <= 0) return cudaSuccess;
-  const dim3 g(grid), b(GEMM_THREADS);
-  if (op == OP_GRAM) {
-    ns_gemm_kernel<OP_GRAM><<<g, b, GEMM_SMEM_BYTES, stream>>>(L);
-  } else if (op == OP_POLY) {
-    ns_gemm_kernel<OP_POLY><<<g, b, GEMM_SMEM_BYTES, stream>>>(L);
-  } else if (L.final_mode == FINAL_NONE) {
-    ns_gemm_kernel<OP_UPDATE><<<g, b, GEMM_SMEM_BYTES, stream>>>(L);
-  } else {
-    ns_gemm_final_kernel<<<g, b, FINAL_SMEM_BYTES, stream>>>(L, *F);
-  }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = (op == OP_UPDATE && L.final_mode != FINAL_NONE) ? FINAL_SMEM_BYTES
+                                                                         : GEMM_SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (op == OP_GRAM) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_GRAM>, L);
+  if (op == OP_POLY) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_POLY>, L);
+  if (L.final_mode == FINAL_NONE) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_UPDATE>, L);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_final_kernel, L, *F);
 }
 
 }  // namespace muon
