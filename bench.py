@@ -261,6 +261,49 @@ def flat_views(torch, shapes, device, dtype, pinned=False):
     return flat, views
 
 
+# ---------------------------------------------------------------- ranks (weak scaling)
+
+class Ranks:
+    """Process-group plumbing of a multi-rank run: every rank times its own
+    independent problem; the only collectives are barriers around the timed
+    region and the max of the per-rank times.  There is no data-path
+    collective.  backend 'nccl' on GPUs, 'gloo' for CPU tests."""
+
+    def __init__(self, world: int, backend: str = "nccl", device=None, timeout_s: int = 120):
+        import torch
+        self.world = world
+        self.device = device if device is not None else torch.device("cpu")
+        self.dist = None
+        if world > 1:
+            import torch.distributed as dist
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.dist is None:
+            return float(v)
+        import torch
+        t = torch.tensor([float(v)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own problem (seed = rank): the step is per-matrix
+    independent, so N ranks run N independent problems (weak scaling)."""
+    return int(rank)
+
+
 def run_ours(args, wl, rank, world):
     import torch
     import newton_schulz_norm_b200 as muon
@@ -268,25 +311,12 @@ def run_ours(args, wl, rank, world):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, "nccl", dev)
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     # ---- inputs (seeded per rank), resident in HBM
-    st = WorkloadStream(wl, seed=rank)
+    st = WorkloadStream(wl, seed=rank_seed(rank))
     params, bufs = st.init()
     grad_sets = [st.next_grads() for _ in range(N_GRAD_SETS)]
 
@@ -421,8 +451,7 @@ def run_ours(args, wl, rank, world):
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
