@@ -114,13 +114,33 @@ def _check_mat(t: torch.Tensor, name: str, dtype=torch.float32):
         raise ValueError(f"{name}: expected a contiguous {dtype} CUDA tensor")
 
 
+def _as_matrix(t: torch.Tensor) -> torch.Tensor:
+    """View an N-D (N >= 3) tensor as (shape[0], prod(shape[1:])) -- a conv
+    weight as its im2col matrix.  1-D tensors are not Muon parameters."""
+    if t.dim() < 2:
+        raise ValueError("Muon updates matrices; 1-D parameters belong to another optimizer")
+    if t.dim() == 2:
+        return t
+    if not t.is_contiguous():
+        raise ValueError("an N-D tensor must be contiguous to be updated through its matrix view")
+    return t.view(t.shape[0], -1)   # a view: the in-place update reaches t
+
+
 def step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
          bufs: Sequence[torch.Tensor], lr: float, beta: float = 0.95, nesterov: bool = True,
-         ns_steps: int = 5, coeffs=DEFAULT_COEFFS, stream=None) -> None:
-    """One Muon step, in place on params and bufs (see include/muon.h)."""
+         ns_steps: int = 5, coeffs=DEFAULT_COEFFS, stream=None, reshape_nd: bool = False) -> None:
+    """One Muon step, in place on params and bufs (see include/muon.h).
+
+    With reshape_nd, tensors of rank >= 3 (conv weights) are updated as their
+    (shape[0], prod(shape[1:])) matrix view; they must be contiguous.
+    """
     n = len(params)
     if len(grads) != n or len(bufs) != n:
         raise ValueError("params, grads and bufs must have the same length")
+    if reshape_nd:
+        params = [_as_matrix(t) for t in params]
+        grads = [_as_matrix(t) for t in grads]
+        bufs = [_as_matrix(t) for t in bufs]
     shapes = []
     for p, g, b in zip(params, grads, bufs):
         for t, nm in ((p, "param"), (g, "grad"), (b, "buf")):

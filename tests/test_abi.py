@@ -90,3 +90,18 @@ def test_workspace_bytes_host_only(lib):
     lower = 2 * 2 * 84934656 + 2 * 2 * 48 * 768 * 768
     assert lower <= b <= lower * 1.05
     assert m.workspace_bytes([(0, 3)]) == -1
+
+
+def test_nd_matrix_view_is_a_view_and_rejects_1d():
+    import torch
+    from newton_schulz_norm_b200 import _as_matrix
+    w = torch.zeros(8, 4, 3, 3)
+    m = _as_matrix(w)
+    assert m.shape == (8, 36) and m.data_ptr() == w.data_ptr()
+    m[2, 5] = 1.0
+    assert w[2, 0, 1, 2] == 1.0          # row-major: 5 = 0*9 + 1*3 + 2
+    assert _as_matrix(torch.zeros(3, 5)).shape == (3, 5)
+    with pytest.raises(ValueError):
+        _as_matrix(torch.zeros(7))
+    with pytest.raises(ValueError):
+        _as_matrix(torch.zeros(4, 8, 3, 3).transpose(0, 1))

@@ -384,3 +384,62 @@ def test_rejects_bad_args_before_launch(muon):
     with pytest.raises(muon.MuonError):
         muon.step([p], [g], [b], lr=0.1, ns_steps=-1)
     assert torch.all(b == 0)
+
+
+def _first_step_sampled(muon, wl, subset_layers, sample):
+    """One step on the listed layers' matrices (all in one call), the oracle on
+    `sample` (indices into the call's matrices)."""
+    idx = [4 * l + k for l in subset_layers for k in range(4)]
+    st = WorkloadStream(wl, seed=0, subset=idx)
+    params, bufs = st.init()
+    grads = st.next_grads()
+    p_d, b_d = _run_step(muon, params, grads, bufs, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov,
+                         ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    assert muon.status() == 0
+    p_ref, b_ref = muon_step_ref([params[i] for i in sample], [grads[i] for i in sample],
+                                 [bufs[i] for i in sample], lr=wl.lr, beta=wl.beta,
+                                 nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    # warm-started momentum: a trajectory step
+    _check_step([params[i] for i in sample], [p_d[i] for i in sample], [b_d[i] for i in sample],
+                p_ref, b_ref, tol=X_TOL_TRAJ)
+
+
+def test_step_gpt2_medium_all_96_sampled(muon):
+    """GPT-2 medium shapes (d = 1024): all 96 matrices in one call."""
+    _first_step_sampled(muon, WORKLOADS["gpt2_medium"], range(24), sample=[0, 1, 2, 3])
+
+
+def test_step_gpt2_xl_two_layers_sampled(muon):
+    """GPT-2 XL shapes (d = 1600, not a multiple of the 256-wide tiles):
+    two layers (8 matrices) in one call, every shape checked."""
+    _first_step_sampled(muon, WORKLOADS["gpt2_xl"], [0, 47], sample=[0, 1, 2, 3, 7])
+
+
+def test_square_8192_closed_form(muon):
+    """The largest square of the sweep, against its known factors."""
+    case = square_case(8192, seed=0)
+    out = to_np(muon.orthogonalize(to_f32(case.g), ns_steps=5))
+    d = case.project(out)
+    target = poly_scalar(case.sigma / np.linalg.norm(case.sigma), COEFFS, 5)
+    assert rel_fro(np.diag(d), target) < 3e-2
+
+
+def test_step_nd_weights_viewed_as_2d(muon):
+    """A conv weight (out, in, kh, kw) is updated as its (out, in*kh*kw) matrix
+    (the im2col view a reply on the X thread asks about)."""
+    rng = _rng(90)
+    shape = (64, 32, 3, 3)
+    p = (rng.standard_normal(shape) * 0.02).astype(np.float32)
+    g = rng.standard_normal(shape).astype(np.float32)
+    b = np.zeros(shape, np.float32)
+    p_d, g_d, b_d = to_f32(p), to_f32(g), to_f32(b)
+    muon.step([p_d], [g_d], [b_d], lr=0.02, reshape_nd=True)
+    torch.cuda.synchronize()
+    p2 = p.reshape(64, -1)
+    p_ref, b_ref = muon_step_ref([p2], [g.reshape(64, -1)], [b.reshape(64, -1)], lr=0.02)
+    _check_step([p2], [p_d.reshape(64, -1)], [b_d.reshape(64, -1)], p_ref, b_ref)
+    with pytest.raises(ValueError):
+        muon.step([p_d], [g_d], [b_d], lr=0.02)           # N-D needs the explicit view
+    one = torch.zeros(16, device="cuda")
+    with pytest.raises(ValueError):
+        muon.step([one], [one], [one], lr=0.02, reshape_nd=True)   # 1-D stays excluded
