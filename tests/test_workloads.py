@@ -56,3 +56,21 @@ def test_square_case_hadamard_factors():
     # H/sqrt(n) is orthogonal
     h = workloads.fwht_rows(np.eye(n)) / np.sqrt(n)
     np.testing.assert_allclose(h @ h.T, np.eye(n), atol=1e-12)
+
+
+def test_adamw_workloads_sizes_and_determinism():
+    from workloads import ADAMW_WORKLOADS, AdamWStream
+    wl = ADAMW_WORKLOADS["gpt2_124m_adamw"]
+    assert wl.n_tensors == 2 + 12 * 8 + 2
+    assert wl.n_elements == 50257 * 768 + 1024 * 768 + 12 * (6 * 768 + 3 * 768 + 4 * 768) + 2 * 768
+    # decay only on the two embeddings (weight decay skips biases and 1-D tensors)
+    assert [t.name for t in wl.tensors if t.decay] == ["wte", "wpe"]
+    small = ADAMW_WORKLOADS["adamw_ragged"]
+    a = AdamWStream(small, seed=3)
+    b = AdamWStream(small, seed=3)
+    for x, y in zip(a.init() + (a.next_grads(),), b.init() + (b.next_grads(),)):
+        for s, t in zip(x, y):
+            assert s.dtype == np.float32
+            np.testing.assert_array_equal(s, t)
+    _, _, vs = AdamWStream(small, seed=0).init()
+    assert all(np.all(v >= 0) for v in vs)

@@ -18,6 +18,16 @@ Workloads (all matrices fp32, row-major, shapes as stored r x c):
 * ``square``       one n x n matrix U diag(sigma) V^T with log-uniform sigma
                    on [1e-3, 1] (condition number 1e3), for the NS-only sweep.
 
+AdamW workloads (the parameters Muon leaves out; fp32 tensors of any rank):
+
+* ``adamw_ragged``     a handful of tensors with ragged sizes (1, 3, 5, 768,
+                       4097, 3x5x7, 50000), some in the no-decay group.
+* ``gpt2_124m_adamw``  the non-hidden parameters of GPT-2 124M: token
+                       embedding 50257x768 and position embedding 1024x768
+                       (decayed), and per block the LayerNorm gains/biases and
+                       the linear biases, plus the final LayerNorm (no decay):
+                       100 tensors, 39,505,152 elements.
+
 GPT-2 dimensions follow "Let's reproduce GPT-2 (124M)" (12 layers, 768
 channels, init std 0.02); the Conv1D weights of GPT-2 are stored transposed
 relative to a linear layer, which is why mlp c_proj is listed 3072x768.
@@ -25,6 +35,9 @@ relative to a linear layer, which is why mlp c_proj is listed 3072x768.
 Draw order (fixed so that a seed names one exact input):
   init   for each matrix in listing order: p, then buf (if warm-started);
   step   for each matrix in listing order: the gradient's factors, then noise.
+  AdamW  init: for each tensor in listing order, p (when drawn), then the
+         gradient average, then the squared-gradient average; step: for each
+         tensor, its gradient.
 """
 from __future__ import annotations
 
@@ -224,3 +237,110 @@ def square_case(n: int, seed: int = 0, cond: float = 1e3) -> SquareCase:
     t = fwht_rows(np.diag(w))             # diag(w) H
     g = fwht_rows(t.T).T / n              # H diag(w) H / n
     return SquareCase(n, sigma, g.astype(np.float32), "hadamard", d1=d1, d2=d2)
+
+
+# ---------------------------------------------------------------- AdamW inputs
+
+@dataclasses.dataclass(frozen=True)
+class AdamWTensor:
+    name: str
+    shape: Tuple[int, ...]
+    decay: bool             # False: the no-decay group (biases, 1-D tensors)
+    init: str               # "normal" (std 0.02), "ones" or "zeros"
+
+    @property
+    def numel(self) -> int:
+        return int(np.prod(self.shape)) if self.shape else 1
+
+
+@dataclasses.dataclass(frozen=True)
+class AdamWWorkload:
+    name: str
+    tensors: Tuple[AdamWTensor, ...]
+    lr: float = 6e-4
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.1
+    step: int = 10          # the step number t of the (first) step drawn
+    grad_std: float = 1e-2
+
+    @property
+    def n_tensors(self) -> int:
+        return len(self.tensors)
+
+    @property
+    def n_elements(self) -> int:
+        return sum(t.numel for t in self.tensors)
+
+
+def _gpt2_adamw_tensors(layers: int, d: int, vocab: int = 50257, ctx: int = 1024):
+    ts = [AdamWTensor("wte", (vocab, d), True, "normal"),
+          AdamWTensor("wpe", (ctx, d), True, "normal")]
+    for l in range(layers):
+        ts += [AdamWTensor(f"h{l}.ln_1.weight", (d,), False, "ones"),
+               AdamWTensor(f"h{l}.ln_1.bias", (d,), False, "zeros"),
+               AdamWTensor(f"h{l}.attn.c_attn.bias", (3 * d,), False, "zeros"),
+               AdamWTensor(f"h{l}.attn.c_proj.bias", (d,), False, "zeros"),
+               AdamWTensor(f"h{l}.ln_2.weight", (d,), False, "ones"),
+               AdamWTensor(f"h{l}.ln_2.bias", (d,), False, "zeros"),
+               AdamWTensor(f"h{l}.mlp.c_fc.bias", (4 * d,), False, "zeros"),
+               AdamWTensor(f"h{l}.mlp.c_proj.bias", (d,), False, "zeros")]
+    ts += [AdamWTensor("ln_f.weight", (d,), False, "ones"),
+           AdamWTensor("ln_f.bias", (d,), False, "zeros")]
+    return tuple(ts)
+
+
+ADAMW_WORKLOADS = {
+    "adamw_ragged": AdamWWorkload("adamw_ragged", (
+        AdamWTensor("a", (1,), True, "normal"),
+        AdamWTensor("b", (3,), False, "normal"),
+        AdamWTensor("c", (5,), True, "normal"),
+        AdamWTensor("d", (768,), False, "ones"),
+        AdamWTensor("e", (4097,), True, "normal"),
+        AdamWTensor("f", (3, 5, 7), True, "normal"),
+        AdamWTensor("g", (50000,), False, "normal"),
+    ), lr=1e-2, step=3),
+    "gpt2_124m_adamw": AdamWWorkload("gpt2_124m_adamw", _gpt2_adamw_tensors(12, 768)),
+}
+
+
+class AdamWStream:
+    """Seeded AdamW state + gradient stream.
+
+    ``init()`` returns fp32 (params, exp_avgs, exp_avg_sqs) as they stand
+    after ``wl.step - 1`` steps: parameters at their GPT-2 initial values
+    (normal std 0.02, LayerNorm gains 1, biases 0), gradient averages
+    N(0, (0.1 grad_std)^2) and squared-gradient averages (grad_std z)^2 with
+    z ~ N(0,1) (non-negative, as a running mean of squares is).  With
+    ``wl.step == 1`` both averages start at zero.  Every ``next_grads()``
+    returns one step's N(0, grad_std^2) gradients.
+    """
+
+    def __init__(self, wl: AdamWWorkload, seed: int = 0):
+        self.wl = wl
+        self.rng = np.random.default_rng(seed)
+
+    def init(self):
+        params, us, vs = [], [], []
+        for t in self.wl.tensors:
+            if t.init == "normal":
+                p = _normal32(self.rng, t.shape, 0.02)
+            elif t.init == "ones":
+                p = np.ones(t.shape, np.float32)
+            else:
+                p = np.zeros(t.shape, np.float32)
+            if self.wl.step > 1:
+                u = _normal32(self.rng, t.shape, 0.1 * self.wl.grad_std)
+                z = _normal32(self.rng, t.shape, self.wl.grad_std)
+                v = z * z
+            else:
+                u = np.zeros(t.shape, np.float32)
+                v = np.zeros(t.shape, np.float32)
+            params.append(p)
+            us.append(u)
+            vs.append(v)
+        return params, us, vs
+
+    def next_grads(self):
+        return [_normal32(self.rng, t.shape, self.wl.grad_std) for t in self.wl.tensors]
