@@ -21,6 +21,11 @@ X-update kernels, grouped over all matrices), and the fused parameter update.
             region, against MEASURED_PEAKS.json.
 * cpu_baseline  the CPU oracle (fp64 NumPy, emulated bf16) on a bounded sample
             (one GPT-2 block, 4 matrices), scaled to the full step.
+* adamw     a side measurement, not part of the step above: one AdamW step
+            over the GPT-2 124M parameters Muon leaves out (embeddings,
+            LayerNorm and bias vectors; 100 tensors, 39.5M elements), timed
+            the same way, with its HBM roofline (28 algorithmic bytes per
+            element).
 
 Under torchrun (N > 1) every rank runs its own independent 48-matrix step on
 its own GPU with its own seed (weak scaling, no data-path collective).
@@ -43,12 +48,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, WorkloadStream  # noqa: E402
+from workloads import ADAMW_WORKLOADS, WORKLOADS, AdamWStream, WorkloadStream  # noqa: E402
 
 METRIC = "Muon step ms, GPT-2 124M 48 mats; Newton-Schulz bf16 TFLOP/s vs tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 N_GRAD_SETS = 4
 KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply")
+ADAMW_BYTES_PER_ELEMENT = 28.0     # read p, g, m, v; write p, m, v (fp32)
 
 
 def parse_args():
@@ -60,6 +66,9 @@ def parse_args():
     ap.add_argument("--workload", default="gpt2_124m", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW side measurement")
+    ap.add_argument("--adamw-only", action="store_true",
+                    help="run only the AdamW side measurement (for profiling that kernel)")
     return ap.parse_args()
 
 
@@ -304,6 +313,70 @@ def rank_seed(rank: int) -> int:
     return int(rank)
 
 
+def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
+    """Time one AdamW step over the non-hidden GPT-2 124M parameters."""
+    import torch
+    import newton_schulz_norm_b200 as muon
+
+    aw = ADAMW_WORKLOADS["gpt2_124m_adamw"]
+    st = AdamWStream(aw, seed=rank_seed(rank))
+    params, us, vs = st.init()
+    grad_sets = [st.next_grads() for _ in range(N_GRAD_SETS)]
+    on_dev = lambda xs: [torch.from_numpy(x).to(dev) for x in xs]  # noqa: E731
+    P, M, V = on_dev(params), on_dev(us), on_dev(vs)
+    G = [on_dev(gs) for gs in grad_sets]
+    decay = [t.decay for t in aw.tensors]
+    kw = dict(lr=aw.lr, betas=(aw.beta1, aw.beta2), eps=aw.eps, weight_decay=aw.weight_decay,
+              decay=decay)
+    for w in range(args.warmup):
+        muon.adamw_step(P, G[w % N_GRAD_SETS], M, V, aw.step + w, **kw)
+    torch.cuda.synchronize()
+    barrier()
+    muon.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    t0 = aw.step + args.warmup
+    for k in range(args.steps):
+        muon.adamw_step(P, G[k % N_GRAD_SETS], M, V, t0 + k, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = muon.profile_end()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    kern_ms, launches = prof["adamw"]
+    per_launch = ADAMW_BYTES_PER_ELEMENT * aw.n_elements   # one launch per step (100 tensors)
+    gbs = per_launch / (kern_ms / launches * 1e-3) / 1e9
+    return {"workload": f"{aw.name}: {aw.n_tensors} fp32 tensors, {aw.n_elements} elements "
+                        f"(wte 50257x768, wpe 1024x768 decayed; LayerNorm and bias vectors not), "
+                        f"lr {aw.lr}, betas ({aw.beta1}, {aw.beta2}), eps {aw.eps}, "
+                        f"weight decay {aw.weight_decay}",
+            "ms_per_step": ms, "launches_per_step": launches / args.steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "bytes_per_launch": per_launch, "avg_launch_ms": kern_ms / launches,
+                         "peak_source": f"{peaks['source']} (burst)"},
+            "l2": f"inputs larger than L2: {N_GRAD_SETS} gradient sets cycled "
+                  f"({N_GRAD_SETS * aw.n_elements * 4 / 1e9:.2f} GB) + 3 state arrays "
+                  f"({3 * aw.n_elements * 4 / 1e9:.2f} GB)"}
+
+
+def run_adamw_only(args, rank, world):
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks(world, "nccl", dev)
+    res = measure_adamw(args, rank, dev, torch.cuda.current_stream(), ranks.barrier, ranks.max,
+                        load_peaks())
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "adamw": res}), flush=True)
+    ranks.close()
+    return 0
+
+
 def run_ours(args, wl, rank, world):
     import torch
     import newton_schulz_norm_b200 as muon
@@ -400,8 +473,11 @@ def run_ours(args, wl, rank, world):
     barrier()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3) / e2e_steps)
 
-    # ---- roofline of the dominant kernel
     peaks = load_peaks()
+    adamw = None if args.no_adamw else measure_adamw(args, rank, dev, stream, barrier,
+                                                      max_over_ranks, peaks)
+
+    # ---- roofline of the dominant kernel
     work = per_launch_work(wl)
     dom = max((k for k in KINDS if prof[k][1] > 0), key=lambda k: prof[k][0])
     bound, per_launch = work[dom]
@@ -448,6 +524,7 @@ def run_ours(args, wl, rank, world):
                 "d2h_bytes_per_step": 4 * wl.n_elements, "steps": e2e_steps},
         "gpu_launches": launches,
         "clocks": clk,
+        "adamw": adamw,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
@@ -462,6 +539,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl, rank)
+    if args.adamw_only:
+        return run_adamw_only(args, rank, world)
     return run_ours(args, wl, rank, world)
 
 

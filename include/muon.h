@@ -168,6 +168,43 @@ MUON_API int muon_momentum_normalize_noalloc(const float* const* grads, float* c
                                              const int64_t* shapes, int n, float beta,
                                              int nesterov, int* dev_status, void* stream);
 
+/*
+ * muon_adamw_step -- one AdamW step over n fp32 tensors of any shape, for the
+ * parameters that the Muon step leaves out (embeddings, LayerNorm gains and
+ * biases, linear biases).  "07. Training neural networks", section "Adam,
+ * weight decay and AdamW", defines it; per element, with t = step:
+ *
+ *   p  <- p * (1 - lr*lambda_i)               decoupled weight decay
+ *   m  <- beta1*m + (1 - beta1)*g             running average of g
+ *   v  <- beta2*v + (1 - beta2)*g*g           running average of g^2
+ *   p  <- p - (lr / (1 - beta1^t)) * m / (sqrt(v / (1 - beta2^t)) + eps)
+ *
+ *   params, grads, exp_avgs (m), exp_avg_sqs (v)
+ *           pointer arrays [n] of fp32 device tensors, contiguous; params,
+ *           exp_avgs and exp_avg_sqs are updated in place, grads read only.
+ *           Before the first step m and v hold zeros.
+ *   numels  host int64 array [n]: elements of each tensor (0 skips it;
+ *           at most 2^40).
+ *   decay   host byte array [n]: non-zero puts tensor i in the decayed group
+ *           (lambda_i = weight_decay), zero in the no-decay group
+ *           (lambda_i = 0); NULL decays every tensor.
+ *   step    t >= 1, the number of this step (bias correction).
+ *   lr >= 0, 0 <= beta1, beta2 < 1, eps >= 0, weight_decay >= 0, all finite;
+ *           taken as doubles; the per-call constants (lr/(1-beta1^t),
+ *           1/sqrt(1-beta2^t), 1-lr*lambda_i) are formed in double on the host
+ *           and rounded once to fp32; the per-element arithmetic is fp32.
+ *   stream  cudaStream_t as void*.
+ * Pointers need only be 4-byte aligned: tensors whose four pointers are all
+ * 16-byte aligned take 16-byte vector accesses, the others scalar ones.
+ * Tensors must not alias one another.  NaN/Inf stay in the elements they
+ * reach.  One kernel launch per 128 tensors; nothing is allocated.
+ */
+MUON_API int muon_adamw_step(float* const* params, const float* const* grads,
+                             float* const* exp_avgs, float* const* exp_avg_sqs,
+                             const int64_t* numels, const unsigned char* decay, int n,
+                             int64_t step, double lr, double beta1, double beta2, double eps,
+                             double weight_decay, void* stream);
+
 /* muon_status -- synchronises the stream, then returns (and clears) the
  * device-side status of the current device: MUON_OK or MUON_ERR_TIMEOUT;
  * MUON_ERR_CUDA if the synchronisation itself failed. */
@@ -194,10 +231,11 @@ MUON_API int64_t muon_workspace_bytes(const int64_t* shapes, int n);
  * time in milliseconds and the launch count:
  *   0 momentum/norm/cast   1 Gram   2 polynomial   3 X update
  *   4 X update with the fused parameter update   5 update without NS steps
+ *   6 AdamW (muon_adamw_step)
  * ms and launches are host arrays of at least nkinds entries.  Returns the
  * number of kinds written, or a negative status.
  */
-#define MUON_PROFILE_KINDS 6
+#define MUON_PROFILE_KINDS 7
 MUON_API void muon_profile_begin(void);
 MUON_API int muon_profile_end(double* ms, int64_t* launches, int nkinds);
 

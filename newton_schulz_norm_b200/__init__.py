@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DEFAULT_COEFFS", "MuonError", "library", "step", "orthogonalize", "momentum_normalize",
     "gram", "poly", "xupdate", "status", "release", "workspace_bytes", "set_wait_limit_ns",
-    "EXPORTS",
+    "adamw_step", "EXPORTS",
 ]
 
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -30,9 +30,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so"
 EXPORTS = ("muon_step", "muon_orthogonalize", "muon_momentum_normalize", "muon_gram", "muon_poly",
            "muon_xupdate", "muon_status", "muon_error_string", "muon_set_wait_limit_ns",
            "muon_workspace_bytes", "muon_release", "muon_version", "muon_profile_begin",
-           "muon_profile_end", "muon_momentum_normalize_noalloc")
+           "muon_profile_end", "muon_momentum_normalize_noalloc", "muon_adamw_step")
 
-PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply")
+PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "adamw")
 
 _STATUS = {0: "MUON_OK", -1: "MUON_ERR_INVALID_ARG", -2: "MUON_ERR_UNSUPPORTED",
            -3: "MUON_ERR_CUDA", -4: "MUON_ERR_NOMEM", -5: "MUON_ERR_TIMEOUT"}
@@ -60,7 +60,7 @@ def library() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(f"{LIB_PATH} is missing: run `python -m newton_schulz_norm_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
-    i, i64, f, u64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64
+    i, i64, f, u64, d = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64, ctypes.c_double
     sig = {
         "muon_step": (i, [_PP, _PP, _PP, _I64P, i, f, f, i, i, _FP, _P]),
         "muon_orthogonalize": (i, [_P, _P, i, i64, i64, i, _FP, _P]),
@@ -77,6 +77,7 @@ def library() -> ctypes.CDLL:
         "muon_profile_begin": (None, []),
         "muon_profile_end": (i, [ctypes.POINTER(ctypes.c_double), _I64P, i]),
         "muon_momentum_normalize_noalloc": (i, [_PP, _PP, _PP, _I64P, _I64P, i, f, i, _P, _P]),
+        "muon_adamw_step": (i, [_PP, _PP, _PP, _PP, _I64P, _P, i, i64, d, d, d, d, d, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -165,6 +166,48 @@ def step_raw(param_ptrs, grad_ptrs, buf_ptrs, shapes, lr, beta=0.95, nesterov=Tr
     return library().muon_step(arr(param_ptrs), arr(grad_ptrs), arr(buf_ptrs), sh, n, float(lr),
                                float(beta), int(bool(nesterov)), int(ns_steps), _coeffs(coeffs),
                                int(stream) if stream is not None else None)
+
+
+def adamw_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+               exp_avgs: Sequence[torch.Tensor], exp_avg_sqs: Sequence[torch.Tensor], step: int,
+               lr: float, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 1e-2,
+               decay: Sequence[bool] | None = None, stream=None) -> None:
+    """One AdamW step, in place on params and both running averages (see
+    include/muon.h).  Tensors: fp32, contiguous, on the GPU, any shape; the
+    four lists match element by element.  ``decay[i]`` false puts tensor i in
+    the no-decay group; ``decay=None`` decays all.  ``step`` counts from 1."""
+    n = len(params)
+    if not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == n):
+        raise ValueError("params, grads, exp_avgs and exp_avg_sqs must have the same length")
+    if decay is not None and len(decay) != n:
+        raise ValueError("decay must have one entry per tensor")
+    numels = []
+    for p, g, m, v in zip(params, grads, exp_avgs, exp_avg_sqs):
+        for t, nm in ((p, "param"), (g, "grad"), (m, "exp_avg"), (v, "exp_avg_sq")):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
+                    or not t.is_contiguous():
+                raise ValueError(f"{nm}: expected a contiguous float32 CUDA tensor")
+        if g.shape != p.shape or m.shape != p.shape or v.shape != p.shape:
+            raise ValueError("param, grad and average shapes differ")
+        numels.append(p.numel())
+    code = adamw_step_raw([t.data_ptr() for t in params], [t.data_ptr() for t in grads],
+                          [t.data_ptr() for t in exp_avgs], [t.data_ptr() for t in exp_avg_sqs],
+                          numels, step, lr, betas, eps, weight_decay, decay, _stream_ptr(stream))
+    _check(code, "muon_adamw_step")
+
+
+def adamw_step_raw(param_ptrs, grad_ptrs, avg_ptrs, sq_ptrs, numels, step, lr, betas=(0.9, 0.999),
+                   eps=1e-8, weight_decay=1e-2, decay=None, stream=0) -> int:
+    """muon_adamw_step on raw device pointers; returns the status code unchanged."""
+    n = len(param_ptrs)
+    arr = lambda xs: (ctypes.c_void_p * max(n, 1))(*xs)  # noqa: E731
+    ne = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in numels])
+    dm = None if decay is None else (ctypes.c_ubyte * max(n, 1))(*[1 if d else 0 for d in decay])
+    return library().muon_adamw_step(arr(param_ptrs), arr(grad_ptrs), arr(avg_ptrs), arr(sq_ptrs), ne,
+                                     ctypes.cast(dm, ctypes.c_void_p) if dm is not None else None, n,
+                                     int(step), float(lr), float(betas[0]), float(betas[1]),
+                                     float(eps), float(weight_decay),
+                                     int(stream) if stream is not None else None)
 
 
 def orthogonalize(x: torch.Tensor, ns_steps: int = 5, coeffs=DEFAULT_COEFFS,

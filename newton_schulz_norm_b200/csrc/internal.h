@@ -161,6 +161,38 @@ struct ApplyLaunch {
   float scale[MUON_MAX_GROUP];
 };
 
+// ---------------------------------------------------------------- AdamW
+// One AdamW step over a list of fp32 tensors of any size: the parameters the
+// Muon step leaves out.  Each tensor is cut into chunks of ADAMW_CHUNK
+// elements; persistent CTAs take chunks in grid-stride order.
+constexpr int ADAMW_THREADS = 256;
+constexpr int ADAMW_VEC = 2;                                   // float4 per array per thread
+constexpr int ADAMW_CHUNK = ADAMW_THREADS * ADAMW_VEC * 4;     // 2048 elements
+constexpr int ADAMW_MAX_TENSORS = 128;                         // per launch
+
+struct AdamWTensor {
+  float* p;
+  const float* g;
+  float* m;                  // running average of the gradient
+  float* v;                  // running average of its square
+  long long numel;           // > 0
+  int chunk0;                // first chunk of this tensor in the launch
+  int vec;                   // all four pointers 16-byte aligned: float4 path
+  float decay;               // fp32(1 - lr * weight_decay_i)
+  int pad_;
+};
+
+struct AdamWLaunch {
+  int n;                     // tensors in this launch
+  int nchunks;               // chunks of all of them
+  float beta1, one_minus_beta1;
+  float beta2, one_minus_beta2;
+  float step_size;           // fp32(lr / (1 - beta1^t))
+  float inv_sqrt_bc2;        // fp32(1 / sqrt(1 - beta2^t))
+  float eps;
+  AdamWTensor t[ADAMW_MAX_TENSORS];
+};
+
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
                            cudaStream_t stream);
@@ -169,5 +201,7 @@ int ns_gemm_max_pairs();
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);
 int k1_blocks_per_sm();
 cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream);
+cudaError_t launch_adamw(const AdamWLaunch& L, int grid, cudaStream_t stream);
+int adamw_blocks_per_sm();
 
 }  // namespace muon

@@ -162,6 +162,7 @@ struct DeviceCtx {
   int device = -1;
   int num_sms = 0;
   int k1_blocks_per_sm = 1;
+  int adamw_blocks_per_sm = 1;
   int max_pairs = 1;           // co-resident CTA pairs of the GEMM kernels
   int* status = nullptr;
   std::map<std::vector<long long>, std::unique_ptr<Plan>> plans;
@@ -171,7 +172,9 @@ struct DeviceCtx {
 std::map<int, std::unique_ptr<DeviceCtx>> g_ctx;
 
 // ---------------------------------------------------------------- profiling events
-enum ProfKind : int { PK_K1 = 0, PK_GRAM = 1, PK_POLY = 2, PK_UPDATE = 3, PK_FINAL = 4, PK_APPLY = 5 };
+enum ProfKind : int {
+  PK_K1 = 0, PK_GRAM = 1, PK_POLY = 2, PK_UPDATE = 3, PK_FINAL = 4, PK_APPLY = 5, PK_ADAMW = 6
+};
 
 struct ProfRecord {
   int kind;
@@ -239,6 +242,7 @@ int get_ctx(DeviceCtx** out) {
   ctx->max_pairs = ns_gemm_max_pairs();
   if (ctx->max_pairs < 1) ctx->max_pairs = std::max(1, prop.multiProcessorCount / 2);
   ctx->k1_blocks_per_sm = k1_blocks_per_sm();   // persistent: as many CTAs as fit
+  ctx->adamw_blocks_per_sm = adamw_blocks_per_sm();
   *out = ctx.get();
   g_ctx[dev] = std::move(ctx);
   return MUON_OK;
@@ -750,6 +754,83 @@ int muon_step(float* const* params, const float* const* grads, float* const* buf
     if (rc) return rc;
   }
   return MUON_OK;
+}
+
+int muon_adamw_step(float* const* params, const float* const* grads, float* const* exp_avgs,
+                    float* const* exp_avg_sqs, const int64_t* numels, const unsigned char* decay,
+                    int n, int64_t step, double lr, double beta1, double beta2, double eps,
+                    double weight_decay, void* stream) {
+  if (n < 0) return MUON_ERR_INVALID_ARG;
+  if (n == 0) return MUON_OK;
+  if (!params || !grads || !exp_avgs || !exp_avg_sqs || !numels) return MUON_ERR_INVALID_ARG;
+  if (step < 1) return MUON_ERR_INVALID_ARG;
+  for (double h : {lr, beta1, beta2, eps, weight_decay})
+    if (!std::isfinite(h)) return MUON_ERR_INVALID_ARG;
+  if (lr < 0 || eps < 0 || weight_decay < 0 || beta1 < 0 || beta1 >= 1 || beta2 < 0 || beta2 >= 1)
+    return MUON_ERR_INVALID_ARG;
+  constexpr long long kMaxNumel = (1ll << 40);
+  int nonempty = 0;
+  for (int i = 0; i < n; ++i) {
+    if (numels[i] < 0 || numels[i] > kMaxNumel) return MUON_ERR_INVALID_ARG;
+    if (numels[i] == 0) continue;
+    ++nonempty;
+    if (!params[i] || !grads[i] || !exp_avgs[i] || !exp_avg_sqs[i]) return MUON_ERR_INVALID_ARG;
+    for (const void* q : {(const void*)params[i], (const void*)grads[i], (const void*)exp_avgs[i],
+                          (const void*)exp_avg_sqs[i]})
+      if (reinterpret_cast<uintptr_t>(q) & 3u) return MUON_ERR_UNSUPPORTED;   // not a float address
+  }
+  if (nonempty == 0) return MUON_OK;
+  // Host-side constants in double, each rounded once to fp32.
+  const double bc1 = 1.0 - std::pow(beta1, (double)step);
+  const double bc2 = 1.0 - std::pow(beta2, (double)step);
+  static thread_local AdamWLaunch L;
+  L.beta1 = (float)beta1;
+  L.one_minus_beta1 = (float)(1.0 - beta1);
+  L.beta2 = (float)beta2;
+  L.one_minus_beta2 = (float)(1.0 - beta2);
+  L.step_size = (float)(lr / bc1);
+  L.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+  L.eps = (float)eps;
+
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int max_grid = ctx->num_sms * ctx->adamw_blocks_per_sm;
+  auto flush = [&]() -> int {
+    if (L.n == 0) return MUON_OK;
+    const int grid = std::max(1, std::min(L.nchunks, max_grid));
+    ProfScope ps(PK_ADAMW, s);
+    const int r = cuda_err(launch_adamw(L, grid, s));
+    L.n = 0;
+    L.nchunks = 0;
+    return r;
+  };
+  L.n = 0;
+  L.nchunks = 0;
+  constexpr long long kMaxChunks = (1ll << 30);
+  for (int i = 0; i < n; ++i) {
+    if (numels[i] == 0) continue;
+    const long long chunks = cdiv(numels[i], ADAMW_CHUNK);
+    if (L.n == ADAMW_MAX_TENSORS || L.nchunks + chunks > kMaxChunks) {
+      rc = flush();
+      if (rc) return rc;
+    }
+    AdamWTensor& T = L.t[L.n++];
+    T.p = params[i];
+    T.g = grads[i];
+    T.m = exp_avgs[i];
+    T.v = exp_avg_sqs[i];
+    T.numel = numels[i];
+    T.chunk0 = L.nchunks;
+    T.vec = aligned16(params[i]) && aligned16(grads[i]) && aligned16(exp_avgs[i]) &&
+            aligned16(exp_avg_sqs[i]);
+    T.decay = (float)(1.0 - lr * ((decay == nullptr || decay[i]) ? weight_decay : 0.0));
+    T.pad_ = 0;
+    L.nchunks += (int)chunks;
+  }
+  return flush();
 }
 
 int muon_orthogonalize(const float* x, void* out, int out_is_bf16, int64_t rows, int64_t cols,

@@ -105,3 +105,28 @@ def test_nd_matrix_view_is_a_view_and_rejects_1d():
         _as_matrix(torch.zeros(7))
     with pytest.raises(ValueError):
         _as_matrix(torch.zeros(4, 8, 3, 3).transpose(0, 1))
+
+
+def test_adamw_argument_checks_without_gpu(lib):
+    P = ctypes.c_void_p
+    arr = (P * 1)(P(16))
+    ne = (ctypes.c_int64 * 1)(10)
+    call = lambda n=1, a=arr, numels=ne, step=1, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0: \
+        lib.muon_adamw_step(a, a, a, a, numels, None, n, step, lr, b1, b2, eps, wd, None)  # noqa: E731
+    assert lib.muon_adamw_step(None, None, None, None, None, None, 0, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0,
+                               None) == 0
+    assert call(n=-1) == -1
+    assert lib.muon_adamw_step(None, arr, arr, arr, ne, None, 1, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0,
+                               None) == -1
+    assert call(step=0) == -1
+    assert call(lr=float("nan")) == -1
+    assert call(lr=-1e-3) == -1
+    assert call(b1=1.0) == -1
+    assert call(b2=-0.1) == -1
+    assert call(eps=float("inf")) == -1
+    assert call(wd=-0.1) == -1
+    assert call(numels=(ctypes.c_int64 * 1)(-5)) == -1
+    assert call(a=(P * 1)(P(None))) == -1                            # null tensor pointer
+    assert call(a=(P * 1)(P(18))) == -2                              # not even float-aligned
+    # empty tensors are skipped before any device work, even with null pointers
+    assert call(a=(P * 1)(P(None)), numels=(ctypes.c_int64 * 1)(0)) == 0
