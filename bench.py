@@ -15,7 +15,9 @@ X-update kernels, grouped over all matrices), and the fused parameter update.
             sets (1.36 GB, larger than L2), so no step reads a warm L2.
 * e2e       the same step through the public API from pinned host memory:
             every step copies its gradients host->device and reads the
-            updated parameters back device->host inside the timed region.
+            updated parameters back device->host inside the timed region; the
+            copies run on their own streams and overlap the optimizer work of
+            the neighbouring steps (PCIe is full duplex).
 * roofline  the dominant kernel (largest share of device time), timed live
             with CUDA events bracketing each of its launches in the timed
             region, against MEASURED_PEAKS.json.
@@ -67,6 +69,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW side measurement")
+    ap.add_argument("--sharded", action="store_true",
+                    help="matrix-sharded step: the ranks split one problem's matrices and "
+                         "all-gather the parameters (strong scaling)")
     ap.add_argument("--adamw-only", action="store_true",
                     help="run only the AdamW side measurement (for profiling that kernel)")
     return ap.parse_args()
@@ -377,6 +382,54 @@ def run_adamw_only(args, rank, world):
     return 0
 
 
+def run_sharded(args, wl, rank, world):
+    """One problem (seed 0 on every rank) split across the ranks by matrix;
+    each rank steps its own matrices, then one NCCL all-gather of the flat
+    parameter buffer.  Strong scaling: the total work is fixed."""
+    import torch
+    from newton_schulz_norm_b200.sharded import ShardedMuon
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks(world, "nccl", dev)
+    st = WorkloadStream(wl, seed=0)
+    params, _ = st.init()
+    grad_sets = [st.next_grads() for _ in range(N_GRAD_SETS)]
+    sm = ShardedMuon(wl.shapes, ns_steps=wl.ns_steps, device=dev)
+    for v, a in zip(sm.params, params):
+        v.copy_(torch.from_numpy(a))
+    G = [[torch.from_numpy(g).to(dev) for g in gs] for gs in grad_sets]
+    kw = dict(lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov, coeffs=wl.coeffs)
+    stream = torch.cuda.current_stream()
+    for w in range(args.warmup):
+        sm.step(G[w % N_GRAD_SETS], **kw)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        sm.step(G[k % N_GRAD_SETS], **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(e0.elapsed_time(e1) / args.steps)
+    owned = len(sm.owned)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "mode": "sharded",
+            "config": dict(workload_config(wl), parallelism=f"matrix-sharded x{world}",
+                           matrices_on_rank0=owned),
+        }), flush=True)
+    ranks.close()
+    return 0
+
+
 def run_ours(args, wl, rank, world):
     import torch
     import newton_schulz_norm_b200 as muon
@@ -459,15 +512,47 @@ def run_ours(args, wl, rank, world):
             t.copy_(torch.from_numpy(a))
         hg.append(f)
     hp, _ = flat_views(torch, shapes, "cpu", torch.float32, pinned=True)
+    p_snap = torch.empty_like(p_flat)
+    # Three streams, so that the copies in and out overlap the optimizer work
+    # of neighbouring steps (PCIe is full duplex): step k's gradients go in
+    # on s_in while step k-1 computes; after step k the updated parameters
+    # are snapshotted on the device (one D2D copy) and the snapshot goes out
+    # on s_out while step k+1 computes.  Gradient buffers alternate between
+    # two device sets.  Every step still copies its own gradients in and its
+    # own parameters out.
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done = [ev() for _ in range(e2e_steps)]
+    step_done = [ev() for _ in range(e2e_steps)]
+    snap_done = [ev() for _ in range(e2e_steps)]
+    out_done = [ev() for _ in range(e2e_steps)]
     torch.cuda.synchronize()
     barrier()
     e2 = torch.cuda.Event(enable_timing=True)
     e3 = torch.cuda.Event(enable_timing=True)
     e2.record(stream)
+    s_in.wait_event(e2)
+    s_out.wait_event(e2)
     for k in range(e2e_steps):
-        g_flats[0].copy_(hg[k % N_GRAD_SETS], non_blocking=True)
-        muon.step(P, G[0], B, **kw)
-        hp.copy_(p_flat, non_blocking=True)
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(step_done[k - 2])      # step k-2 is done reading this set
+            g_flats[b].copy_(hg[k % N_GRAD_SETS], non_blocking=True)
+            in_done[k].record(s_in)
+        stream.wait_event(in_done[k])
+        muon.step(P, G[b], B, **kw)
+        step_done[k].record(stream)
+        if k >= 1:
+            stream.wait_event(out_done[k - 1])      # the snapshot of step k-1 has left
+        p_snap.copy_(p_flat, non_blocking=True)
+        snap_done[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(snap_done[k])
+            hp.copy_(p_snap, non_blocking=True)
+            out_done[k].record(s_out)
+    stream.wait_event(out_done[e2e_steps - 1])
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -521,7 +606,9 @@ def run_ours(args, wl, rank, world):
         "roofline": roofline, "kernels": kernels,
         "cpu_baseline": cpu_base,
         "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * wl.n_elements,
-                "d2h_bytes_per_step": 4 * wl.n_elements, "steps": e2e_steps},
+                "d2h_bytes_per_step": 4 * wl.n_elements, "steps": e2e_steps,
+                "how": "pinned host gradients in and updated parameters out every step, on two "
+                       "copy streams overlapping neighbouring steps' optimizer work"},
         "gpu_launches": launches,
         "clocks": clk,
         "adamw": adamw,
@@ -541,6 +628,8 @@ def main():
         return run_reference(args, wl, rank)
     if args.adamw_only:
         return run_adamw_only(args, rank, world)
+    if args.sharded:
+        return run_sharded(args, wl, rank, world)
     return run_ours(args, wl, rank, world)
 
 
