@@ -128,10 +128,22 @@ def per_launch_work(wl):
     }
 
 
-def source_hash():
+# The sources each kernel's code and launch configuration come from.
+KIND_SOURCES = {
+    "momentum_norm_cast": ("momentum.cu",),
+    "gram": ("ns_gemm.cu",), "poly": ("ns_gemm.cu",), "xupdate": ("ns_gemm.cu",),
+    "xupdate_final": ("ns_gemm.cu",), "apply": ("momentum.cu",),
+    "adamw": ("adamw.cu",),
+}
+_SHARED_SOURCES = ("internal.h", "ptx.cuh", "muon_api.cu")
+
+
+def source_hash(kind):
+    """Hash of the files that define one kernel kind (its .cu file, the
+    shared headers and the host file that configures its launches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "newton_schulz_norm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KIND_SOURCES[kind] + _SHARED_SOURCES):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -139,41 +151,102 @@ def source_hash():
 
 def recorded_traffic(kind):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic_gpt2_124m.txt")
     try:
         with open(path) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    if d.get("source_hash") != source_hash():
-        return None
     ent = d.get("kernels", {}).get(kind)
-    return None if ent is None else float(ent["bytes_per_launch"])
+    if ent is None or ent.get("source_hash") != source_hash(kind):
+        return None
+    return float(ent["bytes_per_launch"])
 
 
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled every 5 ms through NVML
+    (read only) in a background thread.  Only samples taken between
+    ``load_begin()`` and ``load_end()`` (the timed region, while the GPU runs
+    the queued steps) count; falls back to ``nvidia-smi -lms 100``."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
+        self.samples = []            # (sm_mhz, max_mhz, power_w, reasons_mask)
+        self.loaded = False
+        self.thread = None
         self.proc = None
+        self.nvml = None
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", self.gpu_id], stdout=subprocess.PIPE,
-                stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            self.nvml = (pynvml, h)
+        except Exception:
+            self.nvml = None
+        if self.nvml is None:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                    stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+            time.sleep(0.3)
+            return
+        self.stop_flag = False
+
+        def run():
+            nv, h = self.nvml
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            while not self.stop_flag:
+                if self.loaded:
+                    try:
+                        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax,
+                                             nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                             int(get_reasons(h))))
+                    except Exception:
+                        pass
+                time.sleep(0.005)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def load_begin(self):
+        self.loaded = True
+
+    def load_end(self):
+        self.loaded = False
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
+            sm = [x[0] for x in self.samples]
+            reasons = sorted({nm for x in self.samples for nm, bit in self.REASONS if x[3] & bit})
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_min_mhz": min(sm) if sm else None,
+                    "sm_max_mhz": self.samples[0][1] if self.samples else None,
+                    "power_w_max": max(x[2] for x in self.samples) if self.samples else None,
+                    "samples": len(sm), "source": "NVML every 5 ms during the timed region",
+                    "reasons": reasons}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -201,7 +274,8 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(power) if power else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "source": "nvidia-smi -lms 100 around the timed region",
+                "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline
@@ -358,7 +432,7 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
                         f"weight decay {aw.weight_decay}",
             "ms_per_step": ms, "launches_per_step": launches / args.steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("adamw"),
                          "bytes_per_launch": per_launch, "avg_launch_ms": kern_ms / launches,
                          "peak_source": f"{peaks['source']} (burst)"},
             "l2": f"inputs larger than L2: {N_GRAD_SETS} gradient sets cycled "
@@ -488,17 +562,20 @@ def run_ours(args, wl, rank, world):
     barrier()
     torch.cuda.synchronize()
     muon.profile_begin()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    clocks.load_begin()
+    evs[0].record(stream)
     for k in range(args.steps):
         muon.step(P, G[k % N_GRAD_SETS], B, **kw)
-    e1.record(stream)
+        evs[k + 1].record(stream)
     torch.cuda.synchronize()
+    clocks.load_end()
     prof = muon.profile_end()
     barrier()
     clk = clocks.stop()
-    ms_local = e0.elapsed_time(e1) / args.steps
+    ms_local = evs[0].elapsed_time(evs[-1]) / args.steps
+    per_step = sorted(evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps))
+    pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]  # noqa: E731
     ms = max_over_ranks(ms_local)
     if muon.status() != 0:
         raise RuntimeError("device-side error in the timed region")
@@ -603,6 +680,8 @@ def run_ours(args, wl, rank, world):
         "config": dict(workload_config(wl), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "ns_tflops": ns_tflops, "ns_frac_of_peak": ns_tflops / peaks["bf16_tflops"],
         "ns_ms_per_step": ns_ms,
+        "step_ms_percentiles": {"p10": pct(0.1), "median": statistics.median(per_step),
+                                "p90": pct(0.9), "rank": "0"},
         "roofline": roofline, "kernels": kernels,
         "cpu_baseline": cpu_base,
         "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * wl.n_elements,
