@@ -443,3 +443,32 @@ def test_step_nd_weights_viewed_as_2d(muon):
     one = torch.zeros(16, device="cuda")
     with pytest.raises(ValueError):
         muon.step([one], [one], [one], lr=0.02, reshape_nd=True)   # 1-D stays excluded
+
+
+def test_orthogonalize_max_size_rank1_closed_form(muon):
+    """A 16384 x 65536 input (2^30 elements, 4 GB fp32) of rank one, u v^T:
+    along (u^, v^) the iterate is f_k u^ v^T with the scalar sequence of the
+    rank-1 pin (normalised singular value 1: 0.701000, 1.113620, 0.720706,
+    1.089974, 0.696436), so u^T X v^ = 0.696436.  (Entry by entry the output
+    is not rank one: bf16 rounding puts ~1e-5 into each of the other 16383
+    singular directions and five steps multiply such values by up to
+    a^5 = 485, so the check is the projection, which that noise leaves alone.)"""
+    m, n = 16384, 65536
+    rng = _rng(99)
+    u = rng.standard_normal(m)
+    v = rng.standard_normal(n)
+    u /= np.linalg.norm(u)
+    v /= np.linalg.norm(v)
+    ud = torch.from_numpy(u.astype(np.float32)).cuda()
+    vd = torch.from_numpy(v.astype(np.float32)).cuda()
+    g = torch.outer(ud, vd) * 3.0            # any positive scale: the iteration normalises
+    out = muon.orthogonalize(g, ns_steps=5, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    del g
+    assert muon.status() == 0
+    xv = torch.empty(m, dtype=torch.float64, device="cuda")
+    for i in range(0, m, 1024):
+        xv[i:i + 1024] = (out[i:i + 1024].float() @ vd).double()
+    f_est = float(ud.double() @ xv)
+    assert abs(f_est - 0.696436) < 1e-2 * 0.696436
+    assert bool(torch.isfinite(out).all())
