@@ -88,6 +88,12 @@ typedef enum {
  *   stream  cudaStream_t as void*.
  * params, grads and bufs must not alias one another or across matrices.
  * Returns MUON_OK or a negative muon_status_t.
+ * The first call for a shape set (and for a set of parameter pointers)
+ * allocates and fills the library's scratch and tensor maps, with host
+ * copies.  Later calls with the same shapes and parameter pointers enqueue
+ * only one memset and the kernels on the stream, so such a call can be
+ * captured in a CUDA graph; every replay is one more step on the captured
+ * buffers (the binding's capture_step does this).
  */
 MUON_API int muon_step(float* const* params, const float* const* grads, float* const* bufs,
               const int64_t* shapes, int n, float lr, float beta, int nesterov,

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DEFAULT_COEFFS", "MuonError", "library", "step", "orthogonalize", "momentum_normalize",
     "gram", "poly", "xupdate", "status", "release", "workspace_bytes", "set_wait_limit_ns",
-    "adamw_step", "EXPORTS",
+    "adamw_step", "capture_step", "EXPORTS",
 ]
 
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -154,6 +154,32 @@ def step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
                                float(lr), float(beta), int(bool(nesterov)), int(ns_steps),
                                _coeffs(coeffs), _stream_ptr(stream))
     _check(code, "muon_step")
+
+
+def capture_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+                 bufs: Sequence[torch.Tensor], lr: float, beta: float = 0.95,
+                 nesterov: bool = True, ns_steps: int = 5, coeffs=DEFAULT_COEFFS,
+                 reshape_nd: bool = False) -> "torch.cuda.CUDAGraph":
+    """Run one Muon step eagerly, then capture the next one in a CUDA graph.
+
+    The first call for a set of shapes and parameter pointers builds the
+    library's plan and tensor maps (allocation and host copies, which a
+    capture cannot hold); that is why this function performs one real step
+    before capturing.  Every ``replay()`` of the returned graph is one more
+    step on the same tensors: write each step's gradients into ``grads`` in
+    place before replaying.  The graph keeps the hyper-parameters it was
+    captured with.  Launching nothing but kernels and one memset, a replay
+    saves the host work and launch gaps of the eager call.
+    """
+    kw = dict(lr=lr, beta=beta, nesterov=nesterov, ns_steps=ns_steps, coeffs=coeffs,
+              reshape_nd=reshape_nd)
+    step(params, grads, bufs, **kw)
+    torch.cuda.synchronize()
+    _check(status(), "muon_step (before capture)")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(params, grads, bufs, **kw)
+    return graph
 
 
 def step_raw(param_ptrs, grad_ptrs, buf_ptrs, shapes, lr, beta=0.95, nesterov=True, ns_steps=5,

@@ -472,3 +472,17 @@ def test_orthogonalize_max_size_rank1_closed_form(muon):
     f_est = float(ud.double() @ xv)
     assert abs(f_est - 0.696436) < 1e-2 * 0.696436
     assert bool(torch.isfinite(out).all())
+
+
+@pytest.mark.parametrize("co,steps", [((3.4445, -4.7750, 2.0315), 1), ((3.4445, -4.7750, 2.0315), 3),
+                                      ((3.4445, -4.7750, 2.0315), 10),
+                                      ((1.5, -0.5, 0.0), 8),            # cubic Newton-Schulz (c = 0)
+                                      ((1.875, -1.25, 0.375), 6)])      # convergent quintic
+def test_ns_steps_and_coefficient_sweep(muon, co, steps):
+    """The coefficient/step trade-off space: other triples and step counts
+    through the orthogonalisation entry point, against the oracle."""
+    rng = _rng(120 + steps)
+    g = rng.standard_normal((300, 500)).astype(np.float32)
+    ref = orthogonalize_ref(g, steps, co)
+    out = to_np(muon.orthogonalize(to_f32(g), ns_steps=steps, coeffs=co))
+    assert rel_fro(out, ref) <= (X_TOL if steps <= 5 else X_TOL_TRAJ)
