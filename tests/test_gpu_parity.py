@@ -480,9 +480,24 @@ def test_orthogonalize_max_size_rank1_closed_form(muon):
                                       ((1.875, -1.25, 0.375), 6)])      # convergent quintic
 def test_ns_steps_and_coefficient_sweep(muon, co, steps):
     """The coefficient/step trade-off space: other triples and step counts
-    through the orthogonalisation entry point, against the oracle."""
+    through the orthogonalisation entry point, against the oracle.
+
+    Up to five iterations the 1e-2 bar holds as for the default step.  Past
+    five, the singular values sit in the band the map oscillates in, where it
+    contracts them on average (its Lyapunov exponent along an orbit is -0.49
+    for the default triple), so the sorted singular values must still agree
+    to 1e-2; the singular vectors are not contracted (divided differences of
+    p between band values are near 1 in size) and every further iteration
+    adds a fresh set of accumulation-order roundings, about 0.25% of the
+    Frobenius norm, so the entry-wise bar grows by 2.5e-3 per step past five."""
     rng = _rng(120 + steps)
     g = rng.standard_normal((300, 500)).astype(np.float32)
     ref = orthogonalize_ref(g, steps, co)
     out = to_np(muon.orthogonalize(to_f32(g), ns_steps=steps, coeffs=co))
-    assert rel_fro(out, ref) <= (X_TOL if steps <= 5 else X_TOL_TRAJ)
+    err = rel_fro(out, ref)
+    sv_out = np.linalg.svd(out.astype(np.float64), compute_uv=False)
+    sv_ref = np.linalg.svd(np.asarray(ref, np.float64), compute_uv=False)
+    sv_err = rel_fro(sv_out, sv_ref)
+    print(f"coeffs {co} steps {steps}: entry-wise {err:.4f}, singular values {sv_err:.4f}")
+    assert err <= X_TOL + 2.5e-3 * max(0, steps - 5)
+    assert sv_err <= 1e-2
