@@ -127,46 +127,6 @@ __device__ __forceinline__ void symmetrize_block(uint8_t* blk, int lane) {
   }
 }
 
-// Coalesced layout of a 32x32 bf16 block: lane holds row (lane>>2) + 8k,
-// columns (lane&3)*8 .. +7, for k = 0..3 (each instruction covers 8 rows x
-// 64 contiguous bytes).
-__device__ __forceinline__ void load_block(const __nv_bfloat16* src, long long ld, int rbase,
-                                           int col0, int M, int N, int lane, uint4 (&r)[4]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int row = rbase + (lane >> 2) + 8 * k;
-    const int col = col0 + (lane & 3) * 8;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (row < M && col < N) {
-      const __nv_bfloat16* p = src + (long long)row * ld + col;
-      if (col + 8 <= N) {
-        w = __ldg(reinterpret_cast<const uint4*>(p));
-      } else {
-        uint16_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int e = 0; e < 8 && col + e < N; ++e) h[e] = __bfloat16_as_ushort(p[e]);
-        w.x = h[0] | ((uint32_t)h[1] << 16);
-        w.y = h[2] | ((uint32_t)h[3] << 16);
-        w.z = h[4] | ((uint32_t)h[5] << 16);
-        w.w = h[6] | ((uint32_t)h[7] << 16);
-      }
-    }
-    r[k] = w;
-  }
-}
-
-// Coalesced block -> one row per lane (through the warp's staging block).
-__device__ __forceinline__ void block_to_rows(uint16_t* stg, const uint4 (&r)[4], int lane,
-                                              float (&row)[32]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    *reinterpret_cast<uint4*>(stg + ((lane >> 2) + 8 * k) * EPI_LD + (lane & 3) * 8) = r[k];
-  __syncwarp();
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    unpack8(*reinterpret_cast<const uint4*>(stg + lane * EPI_LD + q * 8), row + 8 * q);
-  __syncwarp();
-}
-
 // One bf16 row per lane -> staging block (row-major).
 __device__ __forceinline__ void rows_to_stage(uint16_t* stg, const float (&x)[32], int lane) {
 #pragma unroll
@@ -202,14 +162,6 @@ __device__ __forceinline__ void stage_to_global(const uint16_t* stg, __nv_bfloat
       }
     }
   }
-  __syncwarp();
-}
-
-// One row per lane -> transposed staging block: element (lane, c) is stored
-// at staging (c, lane), so the block then holds rows of the mirror image.
-__device__ __forceinline__ void rows_to_stage_t(uint16_t* stg, const float (&x)[32], int lane) {
-#pragma unroll
-  for (int c = 0; c < 32; ++c) stg[c * EPI_LD + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(x[c]));
   __syncwarp();
 }
 
