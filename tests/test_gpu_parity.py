@@ -501,3 +501,17 @@ def test_ns_steps_and_coefficient_sweep(muon, co, steps):
     print(f"coeffs {co} steps {steps}: entry-wise {err:.4f}, singular values {sv_err:.4f}")
     assert err <= X_TOL + 2.5e-3 * max(0, steps - 5)
     assert sv_err <= 1e-2
+
+
+def test_step_more_matrices_than_one_group(muon):
+    """600 matrices in one call: more than one launch group holds (512), so
+    the call runs as consecutive groups; every matrix is checked."""
+    rng = _rng(130)
+    shapes = [(int(rng.integers(1, 97)), int(rng.integers(1, 97))) for _ in range(600)]
+    ps = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in shapes]
+    gs = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    bs = [(rng.standard_normal(s) * 0.1).astype(np.float32) for s in shapes]
+    p_d, b_d = _run_step(muon, ps, gs, bs, lr=0.02)
+    assert muon.status() == 0
+    p_ref, b_ref = muon_step_ref(ps, gs, bs, lr=0.02)
+    _check_step(ps, p_d, b_d, p_ref, b_ref, tol=X_TOL_TRAJ)
