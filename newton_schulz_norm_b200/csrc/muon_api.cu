@@ -270,22 +270,31 @@ void full_tiles(std::vector<NsTile>& t, int prob, long long m, long long n, int 
     for (long long j0 = 0; j0 < n; j0 += BN) t.push_back({prob, (int)i0, (int)j0, kc});
 }
 
-// K1 work queue: pass 1 of matrix i+1 sits between passes 1 and 2 of matrix i.
-void k1_items(std::vector<K1Item>& items, const std::vector<K1Info>& info) {
+// K1 work queue.  Pass-2 items of a matrix wait until its norm is known,
+// i.e. until every one of its pass-1 items has finished, so they are queued
+// only once `slack` further pass-1 items (of later matrices) have been
+// queued: by the time the persistent CTAs reach them, the matrix's last
+// pass-1 items are done.  Half the number of resident CTAs is about right;
+// much more slack lets g and buf drop out of L2 before pass 2 reads them
+// again.  Pass-2 runs are inserted between single pass-1 items, so they
+// spread evenly through the queue.
+void k1_items(std::vector<K1Item>& items, const std::vector<K1Info>& info, long long slack) {
   const int n = (int)info.size();
-  auto p1 = [&](int i) {
-    for (int t = 0; t < info[i].nitems; ++t) items.push_back({i, t});
-  };
+  std::vector<long long> end1(n);   // pass-1 items queued when matrix i's pass 1 ends
+  long long queued = 0;
+  int next2 = 0;                    // first matrix whose pass 2 is not queued yet
   auto p2 = [&](int i) {
     for (int t = 0; t < info[i].nitems; ++t) items.push_back({i | K1_PASS2, t});
   };
-  if (n == 0) return;
-  p1(0);
-  for (int i = 1; i < n; ++i) {
-    p1(i);
-    p2(i - 1);
+  for (int i = 0; i < n; ++i) {
+    for (int t = 0; t < info[i].nitems; ++t) {
+      items.push_back({i, t});
+      ++queued;
+      while (next2 < i && queued - end1[next2] >= slack) p2(next2++);
+    }
+    end1[i] = queued;
   }
-  p2(n - 1);
+  while (next2 < n) p2(next2++);
 }
 
 std::vector<K1Info> k1_infos(const std::vector<Geom>& geom, const std::vector<long long>& ldx) {
@@ -399,7 +408,8 @@ int upload_phase(NsPhase& ph, char* base, size_t prob_off, size_t tile_off,
 
 // Builds the scratch memory, tensor maps, tile lists and work queue for a
 // shape set.  with_ns=false builds only the first-kernel part.
-int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan>* out) {
+int build_plan(const std::vector<Geom>& geom, bool with_ns, long long k1_slack,
+               std::unique_ptr<Plan>* out) {
   std::unique_ptr<Plan> P(new Plan());
   P->geom = geom;
   const int n = (int)geom.size();
@@ -501,7 +511,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, std::unique_ptr<Plan
   for (int i = 0; i < n; ++i) ldx[i] = geom[i].ldx;
   std::vector<K1Info> info = k1_infos(geom, ldx);
   std::vector<K1Item> items;
-  k1_items(items, info);
+  k1_items(items, info, k1_slack);
   P->k1.n = n;
   P->k1.info = reinterpret_cast<K1Info*>(base + lay.k1info);
   P->k1.items = reinterpret_cast<K1Item*>(base + lay.k1items);
@@ -538,6 +548,12 @@ int check_coeffs(const float* coeffs, float* co) {
   return MUON_OK;
 }
 
+// Pass-1 items queued between a matrix's pass 1 and its pass 2: half the
+// first kernel's resident CTAs.
+long long k1_queue_slack(const DeviceCtx* ctx) {
+  return std::max(1, ctx->num_sms * ctx->k1_blocks_per_sm / 2);
+}
+
 int get_plan(DeviceCtx* ctx, std::vector<long long> key, const std::vector<Geom>& geom, bool with_ns,
              Plan** out) {
   auto it = ctx->plans.find(key);
@@ -546,7 +562,7 @@ int get_plan(DeviceCtx* ctx, std::vector<long long> key, const std::vector<Geom>
     return MUON_OK;
   }
   std::unique_ptr<Plan> P;
-  int rc = build_plan(geom, with_ns, &P);
+  int rc = build_plan(geom, with_ns, k1_queue_slack(ctx), &P);
   if (rc) return rc;
   *out = P.get();
   ctx->plans[key] = std::move(P);

@@ -52,30 +52,57 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocS
 struct SetupArgs {
   int n;
   int nitems;                       // total work items (both passes)
+  long long slack;                  // pass-1 items queued before a matrix's pass 2
   K1Info info[kMaxMats];
 };
 
-// Writes the per-matrix table and the work queue (pass 1 of matrix i+1
-// between passes 1 and 2 of matrix i, as the regular entry point orders it)
-// and clears the counters.  Runs on the caller's stream before the kernel.
+// Writes the per-matrix table and the work queue, in the regular entry
+// point's order (a matrix's pass-2 items follow `slack` further pass-1 items,
+// inserted between single pass-1 items), and clears the counters.  The queue
+// is a list of runs: run s covers queue positions [seg_start[s],
+// seg_start[s+1]) and holds items seg_first[s], ... of matrix seg_mat[s].
+// Runs on the caller's stream before the kernel.
+constexpr int kMaxRuns = 3 * kMaxMats;   // a pass-2 run can split a pass-1 run in two
+
 __global__ void noalloc_setup_kernel(const __grid_constant__ SetupArgs S, NoAllocScratch* scr) {
-  __shared__ int seg_start[2 * kMaxMats + 1];
-  __shared__ int seg_mat[2 * kMaxMats];
+  __shared__ int seg_start[kMaxRuns + 1];
+  __shared__ int seg_mat[kMaxRuns];
+  __shared__ int seg_first[kMaxRuns];
   __shared__ int nseg;
   if (threadIdx.x == 0) {
     int k = 0, at = 0;
-    auto add = [&](int mat) {
+    auto add = [&](int mat, int first, int count) {
+      if (count <= 0) return;
       seg_start[k] = at;
       seg_mat[k] = mat;
-      at += S.info[mat & ~K1_PASS2].nitems;
+      seg_first[k] = first;
+      at += count;
       ++k;
     };
-    add(0);
-    for (int i = 1; i < S.n; ++i) {
-      add(i);
-      add((i - 1) | K1_PASS2);
+    long long end1[kMaxMats];
+    long long queued = 0;
+    int next2 = 0;
+    for (int i = 0; i < S.n; ++i) {
+      const int ni = S.info[i].nitems;
+      int run0 = 0;                  // first pass-1 item of i not yet in a run
+      for (int t = 0; t < ni; ++t) {
+        ++queued;
+        if (next2 < i && queued - end1[next2] >= S.slack) {
+          add(i, run0, t + 1 - run0);   // pass-1 items run0 .. t
+          run0 = t + 1;
+          while (next2 < i && queued - end1[next2] >= S.slack) {
+            add(next2 | K1_PASS2, 0, S.info[next2].nitems);
+            ++next2;
+          }
+        }
+      }
+      add(i, run0, ni - run0);
+      end1[i] = queued;
     }
-    add((S.n - 1) | K1_PASS2);
+    while (next2 < S.n) {
+      add(next2 | K1_PASS2, 0, S.info[next2].nitems);
+      ++next2;
+    }
     seg_start[k] = at;
     nseg = k;
   }
@@ -90,7 +117,7 @@ __global__ void noalloc_setup_kernel(const __grid_constant__ SetupArgs S, NoAllo
     while (s + 1 < nseg && seg_start[s + 1] <= it) ++s;
     K1Item item;
     item.mat = seg_mat[s];
-    item.group = it - seg_start[s];
+    item.group = seg_first[s] + (it - seg_start[s]);
     scr->items[it] = item;
   }
 }
@@ -177,6 +204,7 @@ extern "C" int muon_momentum_normalize_noalloc(const float* const* grads, float*
   int rc = noalloc_device_setup(dev, &scr, &sms, &bps);
   if (rc) return rc;
 
+  S.slack = std::max(1, sms * bps / 2);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int setup_grid = (int)std::min<long long>(64, cdiv_ll(S.nitems, 256));
   noalloc_setup_kernel<<<setup_grid, 256, 0, s>>>(S, scr);
