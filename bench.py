@@ -651,6 +651,18 @@ def run_ours(args, wl, rank, world):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3) / e2e_steps)
+    # The link itself: one step's gradients in, and its parameters out, each alone.
+    e4 = torch.cuda.Event(enable_timing=True)
+    e5 = torch.cuda.Event(enable_timing=True)
+    e6 = torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    g_flats[0].copy_(hg[0], non_blocking=True)
+    e5.record(stream)
+    hp.copy_(p_flat, non_blocking=True)
+    e6.record(stream)
+    torch.cuda.synchronize()
+    link = {"h2d_gbs": 4 * wl.n_elements / (e4.elapsed_time(e5) * 1e-3) / 1e9,
+            "d2h_gbs": 4 * wl.n_elements / (e5.elapsed_time(e6) * 1e-3) / 1e9}
 
     peaks = load_peaks()
     adamw = None if args.no_adamw else measure_adamw(args, rank, dev, stream, barrier,
@@ -707,7 +719,8 @@ def run_ours(args, wl, rank, world):
         "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * wl.n_elements,
                 "d2h_bytes_per_step": 4 * wl.n_elements, "steps": e2e_steps,
                 "how": "pinned host gradients in and updated parameters out every step, on two "
-                       "copy streams overlapping neighbouring steps' optimizer work"},
+                       "copy streams overlapping neighbouring steps' optimizer work",
+                "link": link},
         "gpu_launches": launches,
         "clocks": clk,
         "adamw": adamw,
