@@ -39,6 +39,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -138,14 +139,22 @@ KIND_SOURCES = {
 _SHARED_SOURCES = ("internal.h", "ptx.cuh", "muon_api.cu")
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank space, so that editing a
+    comment does not mark a kernel as changed."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
 def source_hash(kind):
-    """Hash of the files that define one kernel kind (its .cu file, the
+    """Hash of the code that defines one kernel kind (its .cu file, the
     shared headers and the host file that configures its launches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "newton_schulz_norm_b200", "csrc")
     for name in sorted(KIND_SOURCES[kind] + _SHARED_SOURCES):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -126,8 +126,8 @@ struct K1Ptrs {              // per call
   __nv_bfloat16* x0;         // oriented bf16 output
 };
 
-// Work item: pass in bit 31, matrix in bits [16,31), tile in [0,16) would be
-// too small for big matrices, so items are two ints.
+// Work item: a matrix (K1_PASS2 set for its second pass) and a group of
+// K1_GROUP consecutive tiles of it.
 struct K1Item {
   int mat;                   // matrix index; pass 2 items have mat | 0x40000000
   int group;                 // tiles [group * K1_GROUP, +K1_GROUP) of the matrix

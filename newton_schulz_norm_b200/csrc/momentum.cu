@@ -10,17 +10,20 @@
 //   X0   = bf16(u / (nu + 1e-7)), stored transposed when r > c.
 //
 // The norm needs the whole matrix before any element can be cast, so the
-// kernel works in two passes over 64 x 64 tiles, fed by one work queue:
-//   pass 1 (tile): momentum, write buf, partial sum of squares;
-//   pass 2 (tile): wait until the matrix's norm is published, recompute u
+// kernel works in two passes over 64 x 64 tiles, fed by one work queue of
+// items (four tiles each):
+//   pass 1 (item): momentum, write buf, partial sum of squares;
+//   pass 2 (item): wait until the matrix's norm is published, recompute u
 //                  from g and the new buf, scale, cast, (transpose,) store.
-// The queue holds pass 1 of matrix i+1 between passes 1 and 2 of matrix i, so
-// pass 2 normally re-reads g and buf from L2, and only the one matrix whose
-// norm is pending waits.  The last pass-1 tile of a matrix sums the partials
-// in a fixed order (deterministic norm) and publishes it with a release
-// store.  Pass-2 tiles are queued after every pass-1 tile of their matrix, so
-// a waiting CTA only ever waits on CTAs that are already running; the wait is
-// still bounded and reports MUON_ERR_TIMEOUT instead of hanging.
+// The host queues a matrix's pass-2 items about half a wave of CTAs after its
+// last pass-1 item, behind pass-1 items of later matrices: late enough that
+// the norm is usually published when they are reached, early enough that
+// pass 2 re-reads g and buf mostly from L2.  The last pass-1 item of a
+// matrix sums the partials in a fixed order (deterministic norm) and
+// publishes it with a release store.  Pass-2 items are queued after every
+// pass-1 item of their matrix, so a waiting CTA only ever waits on CTAs that
+// have claimed work ahead of it; the wait is still bounded and reports
+// MUON_ERR_TIMEOUT instead of hanging.
 #include "internal.h"
 #include "ptx.cuh"
 
