@@ -10,20 +10,27 @@
 // Newton-Schulz, in bfloat16.)
 //
 // Design: a persistent, warp-specialised kernel per phase that runs every
-// matrix of the phase as one grouped launch.  Per CTA:
+// matrix of the phase as one grouped launch.  CTAs work in pairs (clusters
+// of two on neighbouring SMs, tcgen05 cta_group::2) on 256 x 256 output
+// tiles; CTA r of a pair holds rows [128r, 128r+128) of the A operand and
+// columns [128r, 128r+128) of the B operand.  Per CTA:
 //   warp 0     one thread issues TMA tile loads (64x64 bf16 boxes, 128-byte
-//              swizzle) into a STAGES-deep ring of shared-memory slices;
-//   warp 1     one thread issues tcgen05.mma (M=128, N=256, K=16, fp32
-//              accumulation in TMEM) and commits slices back to the ring;
+//              swizzle, no multicast) into a ring of shared-memory stages;
+//              both CTAs' bytes complete on the leader CTA's barrier;
+//   warp 1     (leader only) one thread issues tcgen05.mma.cta_group::2
+//              (M=256, N=256, K=16, fp32 accumulation in TMEM) and commits
+//              stages back to both CTAs' rings;
 //   warps 2-9  the epilogue: two warps per TMEM lane quarter, each taking
 //              four 32-column chunks of its 32 rows.  A warp reads its chunk
 //              from TMEM (tcgen05.ld, one row per thread), combines it with
-//              the epilogue input, and moves rows <-> coalesced 32x32 blocks
-//              through a private shared-memory block, so every global load
-//              and store is a full-sector, row-contiguous access.  Epilogue
-//              inputs (X or A) are fetched before the accumulator is ready.
+//              the epilogue input (fetched before the accumulator is ready),
+//              writes bf16 rows into a 64-byte-swizzled 32x32 staging block
+//              and stores it with a TMA store.  Symmetric outputs store each
+//              block above the diagonal twice (as itself and mirrored).
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
-// overlap the main loop of the next.  Every wait is bounded.
+// overlap the main loop of the next.  The last update moves the fp32
+// parameter blocks through a per-warp ring of TMA loads and stores instead.
+// Every wait is bounded.
 #include <cstdio>
 
 #include "internal.h"
