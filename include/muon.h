@@ -100,6 +100,33 @@ MUON_API int muon_step(float* const* params, const float* const* grads, float* c
               int ns_steps, const float* coeffs, void* stream);
 
 /*
+ * muon_step_mirrored -- muon_step that also writes every updated parameter
+ * matrix to n_mirrors further destinations, from the epilogue of the last
+ * Newton-Schulz launch (no separate copy or collective).  For a matrix-
+ * sharded step over several GPUs the destinations are the other GPUs'
+ * copies of the parameters (peer memory reachable through unified virtual
+ * addressing with peer access enabled), so the parameter exchange overlaps
+ * the last GEMM tile by tile.  The stores are plain 16-byte global stores,
+ * followed in every writing thread by a system-scope fence; readers of a
+ * destination must be ordered after the call (for other GPUs: a cross-GPU
+ * barrier in stream order).
+ *
+ *   mirrors    host pointer array [n_mirrors * n]: mirrors[k * n + i] is the
+ *              k-th destination of matrix i, fp32 r_i x c_i row-major,
+ *              16-byte aligned, aliasing nothing else in the call.
+ *   n_mirrors  0..MUON_MAX_MIRRORS (0 is plain muon_step).
+ * Other arguments as muon_step.  Needs ns_steps >= 1 and c_i % 4 == 0 for
+ * every matrix (the paths that write the update from shared-memory blocks);
+ * otherwise MUON_ERR_UNSUPPORTED before anything is enqueued.  The first
+ * call with a new set of destination pointers synchronises the stream.
+ */
+#define MUON_MAX_MIRRORS 7
+MUON_API int muon_step_mirrored(float* const* params, const float* const* grads,
+                                float* const* bufs, const int64_t* shapes, int n, float lr,
+                                float beta, int nesterov, int ns_steps, const float* coeffs,
+                                float* const* mirrors, int n_mirrors, void* stream);
+
+/*
  * muon_orthogonalize -- the Newton-Schulz part alone, for one matrix:
  *   out = NS(bf16(x / (||x||_F + 1e-7)))   (orientation handled as above)
  *

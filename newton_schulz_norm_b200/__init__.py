@@ -30,7 +30,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so"
 EXPORTS = ("muon_step", "muon_orthogonalize", "muon_momentum_normalize", "muon_gram", "muon_poly",
            "muon_xupdate", "muon_status", "muon_error_string", "muon_set_wait_limit_ns",
            "muon_workspace_bytes", "muon_release", "muon_version", "muon_profile_begin",
-           "muon_profile_end", "muon_momentum_normalize_noalloc", "muon_adamw_step")
+           "muon_profile_end", "muon_momentum_normalize_noalloc", "muon_adamw_step",
+           "muon_step_mirrored")
 
 PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "adamw")
 
@@ -78,6 +79,7 @@ def library() -> ctypes.CDLL:
         "muon_profile_end": (i, [ctypes.POINTER(ctypes.c_double), _I64P, i]),
         "muon_momentum_normalize_noalloc": (i, [_PP, _PP, _PP, _I64P, _I64P, i, f, i, _P, _P]),
         "muon_adamw_step": (i, [_PP, _PP, _PP, _PP, _I64P, _P, i, i64, d, d, d, d, d, _P]),
+        "muon_step_mirrored": (i, [_PP, _PP, _PP, _I64P, i, f, f, i, i, _FP, _PP, i, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -129,11 +131,17 @@ def _as_matrix(t: torch.Tensor) -> torch.Tensor:
 
 def step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
          bufs: Sequence[torch.Tensor], lr: float, beta: float = 0.95, nesterov: bool = True,
-         ns_steps: int = 5, coeffs=DEFAULT_COEFFS, stream=None, reshape_nd: bool = False) -> None:
+         ns_steps: int = 5, coeffs=DEFAULT_COEFFS, stream=None, reshape_nd: bool = False,
+         mirrors=None) -> None:
     """One Muon step, in place on params and bufs (see include/muon.h).
 
     With reshape_nd, tensors of rank >= 3 (conv weights) are updated as their
     (shape[0], prod(shape[1:])) matrix view; they must be contiguous.
+
+    mirrors: optional list of destinations, each a list with one entry per
+    parameter (a tensor of the same shape, or a raw device address, e.g. of
+    another GPU's copy); the last kernel writes every updated matrix to each
+    of them as well (muon_step_mirrored).
     """
     n = len(params)
     if len(grads) != n or len(bufs) != n:
@@ -150,6 +158,25 @@ def step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
             raise ValueError("param, grad and buf shapes differ")
         shapes += [p.shape[0], p.shape[1]]
     sh = (ctypes.c_int64 * len(shapes))(*shapes)
+    if mirrors:
+        flat = []
+        for dests in mirrors:
+            if len(dests) != n:
+                raise ValueError("every mirror needs one destination per parameter")
+            for t, p in zip(dests, params):
+                if isinstance(t, torch.Tensor):
+                    if t.shape != p.shape or t.dtype != torch.float32 or not t.is_contiguous():
+                        raise ValueError("a mirror tensor must match its parameter (contiguous fp32)")
+                    flat.append(t.data_ptr())
+                else:
+                    flat.append(int(t))
+        mir = (ctypes.c_void_p * len(flat))(*flat)
+        code = library().muon_step_mirrored(
+            _ptr_array(params), _ptr_array(grads), _ptr_array(bufs), sh, n, float(lr), float(beta),
+            int(bool(nesterov)), int(ns_steps), _coeffs(coeffs), mir, len(mirrors),
+            _stream_ptr(stream))
+        _check(code, "muon_step_mirrored")
+        return
     code = library().muon_step(_ptr_array(params), _ptr_array(grads), _ptr_array(bufs), sh, n,
                                float(lr), float(beta), int(bool(nesterov)), int(ns_steps),
                                _coeffs(coeffs), _stream_ptr(stream))

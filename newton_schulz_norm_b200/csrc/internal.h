@@ -96,6 +96,13 @@ struct NsLaunch {
   // NsProblem::slot) over the stored fp32 parameters, 32 x 32 boxes with
   // 128-byte swizzle; nullptr selects the register read-modify-write path.
   const CUtensorMap* pmaps;
+  // Final FINAL_PARAM launch with mirrors only: a device array of
+  // n_mirrors x mirror_stride parameter pointers; entry k * mirror_stride +
+  // slot receives a copy of every updated block of matrix `slot` (the same
+  // layout as the parameter; the pointer may be another GPU's memory).
+  float* const* mirrors;
+  int n_mirrors;
+  int mirror_stride;
   float ca, cb, cc;
   unsigned long long limit_ns;
   int* status;

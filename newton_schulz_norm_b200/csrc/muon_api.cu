@@ -156,6 +156,10 @@ struct Plan {
   // pointers in pmap_for (rebuilt when a call passes other pointers).
   DevBlock pmap_mem;
   std::vector<const void*> pmap_for;
+  // Device table of mirror destinations of the last X update, valid for the
+  // host pointers in mirror_for (rebuilt when a call passes others).
+  DevBlock mirror_mem;
+  std::vector<const void*> mirror_for;
 };
 
 struct DeviceCtx {
@@ -603,9 +607,13 @@ int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, in
 // The Newton-Schulz chain; the last update writes `final_mode` through F
 // (through the parameter tensor maps `pmaps` when given).
 int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mode,
-           const FinalTable* F, cudaStream_t stream, const CUtensorMap* pmaps = nullptr) {
+           const FinalTable* F, cudaStream_t stream, const CUtensorMap* pmaps = nullptr,
+           float* const* mirrors = nullptr, int n_mirrors = 0) {
   NsLaunch L;
   L.pmaps = nullptr;
+  L.mirrors = nullptr;
+  L.n_mirrors = 0;
+  L.mirror_stride = (int)P->geom.size();
   L.ca = co[0];
   L.cb = co[1];
   L.cc = co[2];
@@ -636,6 +644,8 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     L.ntiles = P->upd[par].ntiles;
     L.final_mode = (s == ns_steps - 1) ? final_mode : FINAL_NONE;
     L.pmaps = (s == ns_steps - 1) ? pmaps : nullptr;
+    L.mirrors = (s == ns_steps - 1) ? mirrors : nullptr;
+    L.n_mirrors = (s == ns_steps - 1) ? n_mirrors : 0;
     {
       ProfScope ps(L.final_mode == FINAL_NONE ? PK_UPDATE : PK_FINAL, stream);
       e = launch_ns_gemm(OP_UPDATE, L, F, pair_grid(ctx, L.ntiles), stream);
@@ -706,9 +716,43 @@ int ensure_param_maps(Plan* P, float* const* params, int n, cudaStream_t stream,
   return MUON_OK;
 }
 
+// Uploads the group's mirror table (n_mirrors x n device pointers, row k
+// contiguous) unless the plan already holds the same one.
+int ensure_mirror_table(Plan* P, float* const* tab, int count, cudaStream_t stream,
+                        float* const** out) {
+  *out = nullptr;
+  if (count == 0) return MUON_OK;
+  std::vector<const void*> want(tab, tab + count);
+  if (P->mirror_mem.ptr && P->mirror_for == want) {
+    *out = reinterpret_cast<float* const*>(P->mirror_mem.ptr);
+    return MUON_OK;
+  }
+  // An earlier launch may still read the old table.
+  if (P->mirror_mem.ptr && cudaStreamSynchronize(stream) != cudaSuccess) return MUON_ERR_CUDA;
+  const size_t bytes = sizeof(float*) * (size_t)count;
+  if (P->mirror_mem.bytes < bytes) {
+    if (P->mirror_mem.ptr) {
+      cudaFree(P->mirror_mem.ptr);
+      P->mirror_mem.ptr = nullptr;
+      P->mirror_mem.bytes = 0;
+    }
+    if (cudaMalloc(&P->mirror_mem.ptr, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_NOMEM;
+    }
+    P->mirror_mem.bytes = bytes;
+  }
+  if (cudaMemcpy(P->mirror_mem.ptr, tab, bytes, cudaMemcpyHostToDevice) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  P->mirror_for = want;
+  *out = reinterpret_cast<float* const*>(P->mirror_mem.ptr);
+  return MUON_OK;
+}
+
 int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, float* const* bufs,
                const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
-               const float* co, cudaStream_t stream) {
+               const float* co, cudaStream_t stream, float* const* mirror_tab = nullptr,
+               int n_mirrors = 0) {
   std::vector<Geom> geom = make_geom(shapes, n);
   Plan* P = nullptr;
   int rc = get_plan(ctx, shape_key('S', geom), geom, true, &P);
@@ -732,7 +776,13 @@ int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, 
   const CUtensorMap* pmaps = nullptr;
   rc = ensure_param_maps(P, params, n, stream, &pmaps);
   if (rc) return rc;
-  return run_ns(ctx, P, ns_steps, co, FINAL_PARAM, &F, stream, pmaps);
+  float* const* mirrors = nullptr;
+  if (n_mirrors > 0) {
+    if (pmaps == nullptr) return MUON_ERR_UNSUPPORTED;   // checked by the caller already
+    rc = ensure_mirror_table(P, mirror_tab, n_mirrors * n, stream, &mirrors);
+    if (rc) return rc;
+  }
+  return run_ns(ctx, P, ns_steps, co, FINAL_PARAM, &F, stream, pmaps, mirrors, n_mirrors);
 }
 
 }  // namespace
@@ -742,11 +792,13 @@ using namespace muon;
 
 extern "C" {
 
-int muon_step(float* const* params, const float* const* grads, float* const* bufs,
-              const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
-              const float* coeffs, void* stream) {
+int muon_step_mirrored(float* const* params, const float* const* grads, float* const* bufs,
+                       const int64_t* shapes, int n, float lr, float beta, int nesterov,
+                       int ns_steps, const float* coeffs, float* const* mirrors, int n_mirrors,
+                       void* stream) {
   int rc = check_shapes(shapes, n);
   if (rc) return rc;
+  if (n_mirrors < 0 || n_mirrors > MUON_MAX_MIRRORS) return MUON_ERR_INVALID_ARG;
   if (n == 0) return MUON_OK;
   if (!params || !grads || !bufs) return MUON_ERR_INVALID_ARG;
   if (!std::isfinite(lr) || !std::isfinite(beta)) return MUON_ERR_INVALID_ARG;
@@ -759,17 +811,40 @@ int muon_step(float* const* params, const float* const* grads, float* const* buf
     if (!aligned16(params[i]) || !aligned16(grads[i]) || !aligned16(bufs[i]))
       return MUON_ERR_UNSUPPORTED;
   }
+  if (n_mirrors > 0) {
+    if (!mirrors) return MUON_ERR_INVALID_ARG;
+    for (long long j = 0; j < (long long)n_mirrors * n; ++j) {
+      if (!mirrors[j]) return MUON_ERR_INVALID_ARG;
+      if (!aligned16(mirrors[j])) return MUON_ERR_UNSUPPORTED;
+    }
+    // Mirrors are written from the shared-memory parameter blocks of the
+    // last X update, which need at least one iteration and c % 4 == 0.
+    if (ns_steps < 1) return MUON_ERR_UNSUPPORTED;
+    for (int i = 0; i < n; ++i)
+      if (shapes[2 * i + 1] % 4 != 0) return MUON_ERR_UNSUPPORTED;
+  }
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceCtx* ctx = nullptr;
   rc = get_ctx(&ctx);
   if (rc) return rc;
+  std::vector<float*> tab;
   for (int g0 = 0; g0 < n; g0 += MUON_MAX_GROUP) {
     const int gn = std::min(MUON_MAX_GROUP, n - g0);
+    tab.assign((size_t)n_mirrors * gn, nullptr);
+    for (int k = 0; k < n_mirrors; ++k)
+      for (int i = 0; i < gn; ++i) tab[(size_t)k * gn + i] = mirrors[(size_t)k * n + g0 + i];
     rc = step_group(ctx, params + g0, grads + g0, bufs + g0, shapes + 2 * g0, gn, lr, beta, nesterov,
-                    ns_steps, co, static_cast<cudaStream_t>(stream));
+                    ns_steps, co, static_cast<cudaStream_t>(stream), tab.data(), n_mirrors);
     if (rc) return rc;
   }
   return MUON_OK;
+}
+
+int muon_step(float* const* params, const float* const* grads, float* const* bufs,
+              const int64_t* shapes, int n, float lr, float beta, int nesterov, int ns_steps,
+              const float* coeffs, void* stream) {
+  return muon_step_mirrored(params, grads, bufs, shapes, n, lr, beta, nesterov, ns_steps, coeffs,
+                            nullptr, 0, stream);
 }
 
 int muon_adamw_step(float* const* params, const float* const* grads, float* const* exp_avgs,
@@ -976,6 +1051,9 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
   }
   NsLaunch L;
   L.pmaps = nullptr;
+  L.mirrors = nullptr;
+  L.n_mirrors = 0;
+  L.mirror_stride = 0;
   L.probs = P->poly.probs;
   L.tiles = P->poly.tiles;
   L.ntiles = P->poly.ntiles;

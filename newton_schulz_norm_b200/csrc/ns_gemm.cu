@@ -284,7 +284,45 @@ __device__ __forceinline__ void final_apply(const NsProblem& P, const FinalTable
   __syncwarp();
 }
 
-template <int OP, bool FINAL>
+// Copies one finished 32 x 32 fp32 parameter block (128-byte swizzle: block
+// element (r, c) at r*128 + (((c >> 2) ^ (r & 7)) << 4) + (c & 3)*4) from
+// shared memory to every mirror of its matrix.  Block element (r, c) is
+// parameter element (base_r + r, base_c + c).  Each store instruction of the
+// warp writes four whole 128-byte rows: lane l takes 16-byte chunk l & 7 of
+// rows (l >> 3) + 4k.
+__device__ __forceinline__ void mirror_block(const NsLaunch& L, const NsProblem& P,
+                                             const uint8_t* blk, int base_r, int base_c, int lane) {
+  const int R = P.transposed ? P.N : P.M;   // parameter rows and columns
+  const int C = P.transposed ? P.M : P.N;
+  const int q = lane & 7;
+  const int col = base_c + 4 * q;
+  float4 v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (lane >> 3) + 4 * k;
+    v[k] = *reinterpret_cast<const float4*>(blk + r * 128 + ((q ^ (r & 7)) << 4));
+  }
+  if (col >= C) return;
+  for (int m = 0; m < L.n_mirrors; ++m) {
+    float* dst = L.mirrors[m * L.mirror_stride + P.slot];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int prow = base_r + (lane >> 3) + 4 * k;
+      if (prow >= R) continue;
+      float* d = dst + (long long)prow * P.ld_final + col;
+      if (col + 4 <= C) {
+        *reinterpret_cast<float4*>(d) = v[k];
+      } else {
+        const float e[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (col + j < C) d[j] = e[j];
+      }
+    }
+  }
+}
+
+template <int OP, bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
   constexpr int NST = FINAL ? FINAL_STAGES : STAGES;            // main-loop ring depth
   constexpr int EPI_REGION = FINAL ? FINAL_EPI_BYTES : EPI_STAGE_BYTES;   // per epilogue warp
@@ -580,6 +618,12 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
               if (P.transposed) tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, rb, col0);
               else tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, col0, rb);
             }
+            if constexpr (MIRROR) {
+              // The block is final in shared memory (only read from here on,
+              // by this warp and the TMA store), so the lanes copy it out too.
+              if (P.transposed) mirror_block(L, P, blk, col0, rb, lane);
+              else mirror_block(L, P, blk, rb, col0, lane);
+            }
           }
         }
         if (lane == 0) bulk_commit_group();        // one group per chunk, empty or not
@@ -725,6 +769,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     }
     // Stores must finish reading shared memory (and land) before the CTA exits.
     if (lane == 0) bulk_wait_group_all();
+    if constexpr (MIRROR) __threadfence_system();   // mirror stores, possibly to peers
     __syncwarp();
   }
 
@@ -749,6 +794,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   ns_gemm_body<OP_UPDATE, true>(L, &F);
 }
 
+// The last update that also writes every parameter block to its mirrors.
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    ns_gemm_final_mirror_kernel(const __grid_constant__ NsLaunch L,
+                                const __grid_constant__ FinalTable F) {
+  ns_gemm_body<OP_UPDATE, true, true>(L, &F);
+}
+
 }  // namespace
 
 cudaError_t ns_gemm_setup(int /*device*/) {
@@ -762,8 +814,11 @@ cudaError_t ns_gemm_setup(int /*device*/) {
   e = cudaFuncSetAttribute(ns_gemm_kernel<OP_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)GEMM_SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)FINAL_SMEM_BYTES);
+  e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)FINAL_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ns_gemm_final_mirror_kernel,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FINAL_SMEM_BYTES);
 }
 
 // How many CTA pairs (clusters of two) can be resident at once.
@@ -807,6 +862,11 @@ cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int g
   if (op == OP_GRAM) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_GRAM>, L);
   if (op == OP_POLY) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_POLY>, L);
   if (L.final_mode == FINAL_NONE) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_UPDATE>, L);
+  if (L.n_mirrors > 0) {
+    // Mirrors are written only from the shared-memory parameter ring.
+    if (L.final_mode != FINAL_PARAM || L.pmaps == nullptr) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, ns_gemm_final_mirror_kernel, L, *F);
+  }
   return cudaLaunchKernelEx(&cfg, ns_gemm_final_kernel, L, *F);
 }
 

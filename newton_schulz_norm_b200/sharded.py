@@ -16,6 +16,12 @@ The parameters live in one flat fp32 buffer laid out by owner: rank k's
 matrices are contiguous in segment k, and all segments have the same length,
 so the all-gather writes the buffer in place (NCCL all-gather into a tensor
 whose k-th slice is rank k's input).
+
+With ``fused=True`` (several GPUs) the flat buffer is symmetric memory: every
+rank can address every other rank's copy.  The last kernel of each rank's
+step then writes its updated matrices straight into all the other copies
+(muon_step_mirrored: peer stores from the epilogue, overlapping the last
+GEMM), and a device-side barrier replaces the all-gather.
 """
 from __future__ import annotations
 
@@ -57,6 +63,14 @@ def _round_up(v: int, m: int) -> int:
     return (v + m - 1) // m * m
 
 
+def mirror_pointers(owned: Sequence[int], byte_offsets: Sequence[int], bases: Sequence[int],
+                    rank: int) -> List[List[int]]:
+    """Destinations of this rank's matrices in every other rank's buffer:
+    one list per other rank (in rank order), one address per owned matrix."""
+    return [[int(bases[k]) + int(byte_offsets[i]) for i in owned]
+            for k in range(len(bases)) if k != rank]
+
+
 class ShardedMuon:
     """Muon step partitioned over the ranks of a process group.
 
@@ -68,7 +82,7 @@ class ShardedMuon:
     """
 
     def __init__(self, shapes: Sequence[Tuple[int, int]], group=None, ns_steps: int = 5,
-                 device=None, step_fn: Optional[Callable] = None):
+                 device=None, step_fn: Optional[Callable] = None, fused: bool = False):
         import torch.distributed as dist
 
         self.shapes = [(int(r), int(c)) for r, c in shapes]
@@ -94,12 +108,27 @@ class ShardedMuon:
             offs[i] = seg_len[k]
             seg_len[k] = _round_up(seg_len[k] + r * c, _ALIGN)
         self.seg = max(max(seg_len), _ALIGN)
-        self.flat = torch.zeros(self.world * self.seg, dtype=torch.float32, device=device)
+        self.owned = [i for i in range(len(self.shapes)) if self.owner[i] == self.rank]
+        self.fused = bool(fused) and self.world > 1
+        self._symm = None
+        self._mirrors = None
+        if self.fused:
+            import torch.distributed._symmetric_memory as symm_mem
+            pg = group if group is not None else dist.group.WORLD
+            self.flat = symm_mem.empty(self.world * self.seg, dtype=torch.float32, device=device)
+            self.flat.zero_()
+            self._symm = symm_mem.rendezvous(self.flat, pg)
+        else:
+            self.flat = torch.zeros(self.world * self.seg, dtype=torch.float32, device=device)
         self.params: List[torch.Tensor] = []
+        starts = []
         for i, (r, c) in enumerate(self.shapes):
             base = self.owner[i] * self.seg + offs[i]
+            starts.append(base)
             self.params.append(self.flat[base:base + r * c].view(r, c))
-        self.owned = [i for i in range(len(self.shapes)) if self.owner[i] == self.rank]
+        if self.fused:
+            self._mirrors = mirror_pointers(self.owned, [4 * b for b in starts],
+                                            list(self._symm.buffer_ptrs), self.rank)
         # momentum only for the matrices this rank steps
         self.bufs = {i: torch.zeros(self.shapes[i], dtype=torch.float32, device=device)
                      for i in self.owned}
@@ -118,9 +147,14 @@ class ShardedMuon:
                 kw["coeffs"] = coeffs
             if stream is not None:
                 kw["stream"] = stream
+            if self.fused:
+                kw["mirrors"] = self._mirrors
             self.step_fn([self.params[i] for i in self.owned], [grads[i] for i in self.owned],
                          [self.bufs[i] for i in self.owned], **kw)
-        self.gather()
+        if self.fused:
+            self._symm.barrier()     # every rank's peer stores are done and visible
+        else:
+            self.gather()
 
     def gather(self) -> None:
         """Every rank's segment to every rank (in place in the flat buffer)."""

@@ -130,3 +130,19 @@ def test_adamw_argument_checks_without_gpu(lib):
     assert call(a=(P * 1)(P(18))) == -2                              # not even float-aligned
     # empty tensors are skipped before any device work, even with null pointers
     assert call(a=(P * 1)(P(None)), numels=(ctypes.c_int64 * 1)(0)) == 0
+
+
+def test_mirrored_step_argument_checks_without_gpu(lib):
+    P = ctypes.c_void_p
+    arr = (P * 1)(P(16))
+    sh = (ctypes.c_int64 * 2)(4, 8)
+    mir = (P * 1)(P(32))
+    f = lib.muon_step_mirrored
+    assert f(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, mir, 8, None) == -1      # > MUON_MAX_MIRRORS
+    assert f(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, None, 1, None) == -1     # no table
+    assert f(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, (P * 1)(P(None)), 1, None) == -1
+    assert f(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 5, None, (P * 1)(P(40)), 1, None) == -2   # misaligned
+    assert f(arr, arr, arr, sh, 1, 0.1, 0.9, 1, 0, None, mir, 1, None) == -2      # needs an iteration
+    odd = (ctypes.c_int64 * 2)(4, 6)
+    assert f(arr, arr, arr, odd, 1, 0.1, 0.9, 1, 5, None, mir, 1, None) == -2     # c % 4 != 0
+    assert f(None, None, None, None, 0, 0.1, 0.9, 1, 5, None, None, 0, None) == 0  # n = 0

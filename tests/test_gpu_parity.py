@@ -515,3 +515,28 @@ def test_step_more_matrices_than_one_group(muon):
     assert muon.status() == 0
     p_ref, b_ref = muon_step_ref(ps, gs, bs, lr=0.02)
     _check_step(ps, p_d, b_d, p_ref, b_ref, tol=X_TOL_TRAJ)
+
+
+@pytest.mark.parametrize("n_mats", [4, 520])
+def test_step_mirrored_writes_every_destination(muon, n_mats):
+    """muon_step_mirrored: the parameters come out exactly as from muon_step,
+    and every mirror holds them too (520 matrices: two launch groups)."""
+    rng = _rng(140 + n_mats)
+    if n_mats == 4:
+        shapes = [(256, 768), (768, 256), (300, 200), (129, 260)]
+    else:
+        shapes = [(int(rng.integers(1, 97)), 4 * int(rng.integers(1, 25))) for _ in range(n_mats)]
+    ps = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in shapes]
+    gs = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    bs = [(rng.standard_normal(s) * 0.1).astype(np.float32) for s in shapes]
+    p_ref, b_ref = _run_step(muon, ps, gs, bs, lr=0.02)
+    p_d = [to_f32(p) for p in ps]
+    b_d = [to_f32(b) for b in bs]
+    mirrors = [[torch.full(s, float("nan"), device="cuda") for s in shapes] for _ in range(2)]
+    muon.step(p_d, [to_f32(g) for g in gs], b_d, lr=0.02, mirrors=mirrors)
+    torch.cuda.synchronize()
+    assert muon.status() == 0
+    for i in range(n_mats):
+        assert torch.equal(p_d[i], p_ref[i]) and torch.equal(b_d[i], b_ref[i])
+        for dests in mirrors:
+            assert torch.equal(dests[i], p_d[i])

@@ -115,3 +115,12 @@ def test_single_process_layout_without_group():
     g = [torch.ones(s) for s in shapes]
     sm.step(g, lr=1.0, beta=0.0)
     assert all(float(p.sum()) == -p.numel() for p in sm.params)
+
+
+def test_mirror_pointers_address_every_other_rank():
+    from newton_schulz_norm_b200.sharded import mirror_pointers
+    bases = [1 << 40, 2 << 40, 3 << 40]
+    offs = [0, 256, 4096, 8192]
+    got = mirror_pointers([1, 3], offs, bases, rank=1)
+    assert got == [[bases[0] + 256, bases[0] + 8192], [bases[2] + 256, bases[2] + 8192]]
+    assert mirror_pointers([0], offs, bases[:1], rank=0) == []
