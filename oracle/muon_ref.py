@@ -36,7 +36,7 @@ closed form, diagonal inputs, brute force on 2x2/4x4, invariances).
 from __future__ import annotations
 
 import math
-from typing import List, Sequence, Tuple
+from typing import Sequence, Tuple
 
 import numpy as np
 

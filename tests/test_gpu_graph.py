@@ -1,6 +1,5 @@
 """One Muon step captured in a CUDA graph (capture_step) replays exactly the
 eager step: same kernels, same pointers, bit-identical results."""
-import numpy as np
 import pytest
 import torch
 

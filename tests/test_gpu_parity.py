@@ -31,11 +31,11 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (bf16_round, coeffs_f32, momentum_ref, muon_step_ref, newton_schulz_ref,
-                    normalize_ref, orient, orthogonalize_ref)
+from oracle import (coeffs_f32, momentum_ref, muon_step_ref, newton_schulz_ref, normalize_ref,
+                    orient, orthogonalize_ref)
 from tests.gpu_util import (bf16_agreement, bf16_close, fp32_gemm_bound, rel_fro, to_bf16, to_f32,
                             to_np)
-from tests.spectral import closed_form_ns, lift_threshold, poly_scalar
+from tests.spectral import lift_threshold, poly_scalar
 from workloads import WORKLOADS, WorkloadStream, square_case
 
 pytestmark = pytest.mark.gpu

@@ -4,7 +4,6 @@ muon.step over all matrices gives."""
 import os
 import socket
 
-import numpy as np
 import pytest
 import torch
 

@@ -42,7 +42,6 @@ Draw order (fixed so that a seed names one exact input):
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import List, Sequence, Tuple
 
 import numpy as np
