@@ -570,6 +570,8 @@ def run_ours(args, wl, rank, world):
     # launch.  That bracketing costs about 4% of a step, so the headline pass
     # below runs the same K steps without it.  The two passes are separated by
     # a short idle pause so that each starts from the same power state.
+    torch.cuda.synchronize()
+    time.sleep(0.25)
     barrier()
     torch.cuda.synchronize()
     muon.profile_begin()
