@@ -418,8 +418,10 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
     decay = [t.decay for t in aw.tensors]
     kw = dict(lr=aw.lr, betas=(aw.beta1, aw.beta2), eps=aw.eps, weight_decay=aw.weight_decay,
               decay=decay)
+    # one prepared group per gradient set: arguments checked and packed once
+    groups = [muon.AdamWGroup(P, G[i], M, V, **kw) for i in range(N_GRAD_SETS)]
     for w in range(args.warmup):
-        muon.adamw_step(P, G[w % N_GRAD_SETS], M, V, aw.step + w, **kw)
+        groups[w % N_GRAD_SETS].step(aw.step + w)
     torch.cuda.synchronize()
     barrier()
     muon.profile_begin()
@@ -428,7 +430,7 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
     e0.record(stream)
     t0 = aw.step + args.warmup
     for k in range(args.steps):
-        muon.adamw_step(P, G[k % N_GRAD_SETS], M, V, t0 + k, **kw)
+        groups[k % N_GRAD_SETS].step(t0 + k)
     e1.record(stream)
     torch.cuda.synchronize()
     prof = muon.profile_end()

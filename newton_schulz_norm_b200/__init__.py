@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DEFAULT_COEFFS", "MuonError", "library", "step", "orthogonalize", "momentum_normalize",
     "gram", "poly", "xupdate", "status", "release", "workspace_bytes", "set_wait_limit_ns",
-    "adamw_step", "capture_step", "EXPORTS",
+    "adamw_step", "AdamWGroup", "capture_step", "EXPORTS",
 ]
 
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -247,6 +247,52 @@ def adamw_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
                           [t.data_ptr() for t in exp_avgs], [t.data_ptr() for t in exp_avg_sqs],
                           numels, step, lr, betas, eps, weight_decay, decay, _stream_ptr(stream))
     _check(code, "muon_adamw_step")
+
+
+class AdamWGroup:
+    """A fixed set of AdamW tensors, checked and marshalled once.
+
+    ``adamw_step`` validates and packs every tensor on every call (tens of
+    microseconds of host time for a hundred tensors); a training loop that
+    steps the same tensors each time can build the argument arrays once and
+    then call ``step(t)``, which only passes them on.  The tensors must stay
+    allocated (and at the same addresses) for the group's lifetime.
+    """
+
+    def __init__(self, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+                 exp_avgs: Sequence[torch.Tensor], exp_avg_sqs: Sequence[torch.Tensor],
+                 lr: float, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 1e-2,
+                 decay: Sequence[bool] | None = None):
+        n = len(params)
+        if not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == n):
+            raise ValueError("params, grads, exp_avgs and exp_avg_sqs must have the same length")
+        if decay is not None and len(decay) != n:
+            raise ValueError("decay must have one entry per tensor")
+        for p, g, m, v in zip(params, grads, exp_avgs, exp_avg_sqs):
+            for t, nm in ((p, "param"), (g, "grad"), (m, "exp_avg"), (v, "exp_avg_sq")):
+                if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
+                        or not t.is_contiguous():
+                    raise ValueError(f"{nm}: expected a contiguous float32 CUDA tensor")
+            if g.shape != p.shape or m.shape != p.shape or v.shape != p.shape:
+                raise ValueError("param, grad and average shapes differ")
+        self._keep = (list(params), list(grads), list(exp_avgs), list(exp_avg_sqs))
+        self._n = n
+        arr = lambda ts: (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in ts])  # noqa: E731
+        self._p, self._g, self._m, self._v = (arr(ts) for ts in self._keep)
+        self._numels = (ctypes.c_int64 * max(n, 1))(*[p.numel() for p in params])
+        self._decay = None if decay is None else \
+            (ctypes.c_ubyte * max(n, 1))(*[1 if d else 0 for d in decay])
+        self.lr, self.betas, self.eps, self.weight_decay = float(lr), tuple(betas), float(eps), \
+            float(weight_decay)
+
+    def step(self, step: int, lr: float | None = None, stream=None) -> None:
+        """One AdamW step (t = ``step``, from 1) on the group's tensors."""
+        code = library().muon_adamw_step(
+            self._p, self._g, self._m, self._v, self._numels,
+            ctypes.cast(self._decay, ctypes.c_void_p) if self._decay is not None else None,
+            self._n, int(step), self.lr if lr is None else float(lr), float(self.betas[0]),
+            float(self.betas[1]), self.eps, self.weight_decay, _stream_ptr(stream))
+        _check(code, "muon_adamw_step")
 
 
 def adamw_step_raw(param_ptrs, grad_ptrs, avg_ptrs, sq_ptrs, numels, step, lr, betas=(0.9, 0.999),

@@ -224,3 +224,26 @@ def test_binding_rejects_bad_tensors(muon):
         muon.adamw_step([a], [a], [a], [a.double()], 1, 1e-3)
     with pytest.raises(muon.MuonError):
         muon.adamw_step([a], [a], [a], [a], 0, 1e-3)                # t counts from 1
+
+
+def test_prepared_group_equals_adamw_step(muon):
+    """AdamWGroup (arguments packed once) gives exactly adamw_step's result."""
+    wl = ADAMW_WORKLOADS["adamw_ragged"]
+    st = AdamWStream(wl, seed=5)
+    params, us, vs = st.init()
+    grads = [st.next_grads() for _ in range(3)]
+    decay = [t.decay for t in wl.tensors]
+    kw = dict(lr=wl.lr, betas=(wl.beta1, wl.beta2), eps=wl.eps, weight_decay=wl.weight_decay,
+              decay=decay)
+    a = [_dev(params), _dev(us), _dev(vs)]
+    b = [_dev(params), _dev(us), _dev(vs)]
+    gb = _dev(grads[0])
+    group = muon.AdamWGroup(b[0], gb, b[1], b[2], **kw)
+    for k, gs in enumerate(grads):
+        muon.adamw_step(a[0], _dev(gs), a[1], a[2], wl.step + k, **kw)
+        for d, h in zip(gb, gs):
+            d.copy_(torch.from_numpy(h))
+        group.step(wl.step + k)
+    torch.cuda.synchronize()
+    for x, y in zip(a[0] + a[1] + a[2], b[0] + b[1] + b[2]):
+        assert torch.equal(x, y)
