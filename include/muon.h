@@ -93,7 +93,12 @@ typedef enum {
  * copies.  Later calls with the same shapes and parameter pointers enqueue
  * only one memset and the kernels on the stream, so such a call can be
  * captured in a CUDA graph; every replay is one more step on the captured
- * buffers (the binding's capture_step does this).
+ * buffers (the binding's capture_step does this).  The tensor maps of the
+ * last 8 parameter-pointer sets of a shape set stay cached, so alternating
+ * between up to 8 parameter copies of one shape set neither rebuilds them nor
+ * synchronises; a 9th set evicts the least recently used one after
+ * synchronising the stream (a CUDA graph captured with the evicted set must
+ * not be replayed after that).
  */
 MUON_API int muon_step(float* const* params, const float* const* grads, float* const* bufs,
               const int64_t* shapes, int n, float lr, float beta, int nesterov,
@@ -271,6 +276,19 @@ MUON_API int64_t muon_workspace_bytes(const int64_t* shapes, int n);
 #define MUON_PROFILE_KINDS 7
 MUON_API void muon_profile_begin(void);
 MUON_API int muon_profile_end(double* ms, int64_t* launches, int nkinds);
+
+/*
+ * muon_guard_check -- a check that no kernel wrote outside the scratch
+ * regions it was given (this library's stand-in for a memory checker, which
+ * it does not need a GPU tool for).  Every region of a cached plan (bf16
+ * iterates, Gram and polynomial matrices, problem and tile tables, work
+ * queue, counters, norm partials) is followed by a 256-byte guard band of a
+ * fixed pattern, written when the plan is built and never written by any
+ * kernel.  This call synchronises the current device and returns the number
+ * of guard bytes that no longer hold the pattern, over every plan cached on
+ * that device (0: intact), or a negative status.
+ */
+MUON_API int64_t muon_guard_check(void);
 
 /* muon_release -- synchronises the device and frees every cached plan and
  * scratch buffer of every device this process used. */

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DEFAULT_COEFFS", "MuonError", "library", "step", "orthogonalize", "momentum_normalize",
     "gram", "poly", "xupdate", "status", "release", "workspace_bytes", "set_wait_limit_ns",
-    "adamw_step", "AdamWGroup", "capture_step", "EXPORTS",
+    "adamw_step", "AdamWGroup", "capture_step", "EXPORTS", "guard_check",
 ]
 
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -31,7 +31,7 @@ EXPORTS = ("muon_step", "muon_orthogonalize", "muon_momentum_normalize", "muon_g
            "muon_xupdate", "muon_status", "muon_error_string", "muon_set_wait_limit_ns",
            "muon_workspace_bytes", "muon_release", "muon_version", "muon_profile_begin",
            "muon_profile_end", "muon_momentum_normalize_noalloc", "muon_adamw_step",
-           "muon_step_mirrored")
+           "muon_step_mirrored", "muon_guard_check")
 
 PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "adamw")
 
@@ -80,6 +80,7 @@ def library() -> ctypes.CDLL:
         "muon_momentum_normalize_noalloc": (i, [_PP, _PP, _PP, _I64P, _I64P, i, f, i, _P, _P]),
         "muon_adamw_step": (i, [_PP, _PP, _PP, _PP, _I64P, _P, i, i64, d, d, d, d, d, _P]),
         "muon_step_mirrored": (i, [_PP, _PP, _PP, _I64P, i, f, f, i, i, _FP, _PP, i, _P]),
+        "muon_guard_check": (i64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -400,6 +401,12 @@ def xupdate(b: torch.Tensor, x: torch.Tensor, ca: float) -> torch.Tensor:
 def status(stream=None) -> int:
     """Synchronise and return (and clear) the device-side status code."""
     return library().muon_status(_stream_ptr(stream))
+
+
+def guard_check() -> int:
+    """Synchronise and return how many guard-band bytes around the library's
+    scratch regions were overwritten (0: no kernel wrote out of bounds)."""
+    return int(library().muon_guard_check())
 
 
 def release() -> None:

@@ -10,6 +10,18 @@
 
 namespace muon {
 
+// Built with -DMUON_BOUNDS_CHECK (newton_schulz_norm_b200.build, checked=True),
+// every kernel validates the indices it reads from its tables (tile lists,
+// problem and work-item tables) against the sizes it was launched with before
+// using them; an invalid entry records MUON_ERR_INVALID_ARG in the status
+// word and the work it names is skipped, so a corrupted table becomes an
+// error status instead of an access out of bounds.
+#ifdef MUON_BOUNDS_CHECK
+constexpr bool kBoundsCheck = true;
+#else
+constexpr bool kBoundsCheck = false;
+#endif
+
 // ---------------------------------------------------------------- NS GEMM tiling
 // A CTA pair (cluster of 2, tcgen05 cta_group::2) computes a TILE_M x BN
 // output tile with M=256, N=256, K=16 MMAs issued by the pair's leader:
@@ -91,6 +103,7 @@ struct NsLaunch {
   const NsProblem* probs;
   const NsTile* tiles;
   int ntiles;
+  int nprobs;                // entries of probs (checked builds validate tile.prob)
   int final_mode;
   // Final FINAL_PARAM launch only: one tensor map per matrix (indexed by
   // NsProblem::slot) over the stored fp32 parameters, 32 x 32 boxes with
@@ -145,6 +158,8 @@ struct K1Launch {
   const K1Info* info;
   const K1Item* items;
   int nitems;
+  int n;                     // matrices (entries of info and ptrs)
+  int npartials;             // entries of partials
   int mode;
   int nesterov;
   float beta;
@@ -210,5 +225,8 @@ int k1_blocks_per_sm();
 cudaError_t launch_apply(const ApplyLaunch& L, cudaStream_t stream);
 cudaError_t launch_adamw(const AdamWLaunch& L, int grid, cudaStream_t stream);
 int adamw_blocks_per_sm();
+// The bound of every device-side wait, in ns (muon_set_wait_limit_ns, else
+// MUON_SPIN_LIMIT_NS at first use, else 2 s).  Takes the interface's lock.
+unsigned long long current_wait_limit_ns();
 
 }  // namespace muon

@@ -258,6 +258,20 @@ __global__ void __launch_bounds__(K1_THREADS, 4) k1_kernel(const __grid_constant
     const K1Item item = L.items[it];
     const bool pass2 = (item.mat & K1_PASS2) != 0;
     const int mat = item.mat & ~K1_PASS2;
+    if (kBoundsCheck) {
+      // Checked builds: the item must name a matrix of the launch and one of
+      // its groups, whose partial sum lies inside the partials array.
+      bool ok = mat >= 0 && mat < L.n;
+      if (ok) {
+        const K1Info& q = L.info[mat];
+        ok = item.group >= 0 && item.group < q.nitems && q.part0 >= 0 &&
+             (long long)q.part0 + q.nitems <= L.npartials;
+      }
+      if (!ok) {
+        if (tid == 0) atomicCAS(L.status, 0, MUON_ERR_INVALID_ARG);
+        continue;
+      }
+    }
     const K1Info info = L.info[mat];
     const K1Ptrs P = L.ptrs[mat];
     const int t0 = item.group * K1_GROUP;

@@ -19,6 +19,9 @@
 #include <vector>
 
 #include "internal.h"
+#ifdef MUON_BOUNDS_CHECK
+#include "muon_debug.h"
+#endif
 
 namespace muon {
 namespace {
@@ -102,12 +105,23 @@ bool make_param_map(CUtensorMap* map, const void* base, long long rows, long lon
 
 // ---------------------------------------------------------------- device memory arena
 
+// Guard bands: every region a plan hands out is followed by kGuardBytes of
+// a fixed byte pattern, written when the plan is built and never touched by
+// any kernel.  muon_guard_check() reads them back: a changed byte means some
+// kernel wrote past the end of a region.
+constexpr size_t kGuardBytes = 256;
+constexpr unsigned char kGuardByte = 0xA5;
+
 struct Arena {
   size_t off = 0;
+  std::vector<size_t> guards;   // offsets of the guard bands
   size_t take(size_t bytes, size_t align = 256) {
     off = (off + align - 1) / align * align;
     size_t at = off;
     off += bytes;
+    off = (off + 255) / 256 * 256;
+    guards.push_back(off);
+    off += kGuardBytes;
     return at;
   }
 };
@@ -141,6 +155,7 @@ struct K1Plan {
   double* partials = nullptr;
   double* norms = nullptr;
   int n = 0;
+  int npartials = 0;
 };
 
 struct Plan {
@@ -152,10 +167,14 @@ struct Plan {
   __nv_bfloat16* B = nullptr;
   NsPhase gram[2], poly, upd[2];
   K1Plan k1;
-  // Parameter tensor maps of the last X update, valid for the parameter
-  // pointers in pmap_for (rebuilt when a call passes other pointers).
-  DevBlock pmap_mem;
-  std::vector<const void*> pmap_for;
+  std::vector<size_t> guards;                // guard band offsets in mem
+  // Parameter tensor maps of the last X update, one device block per set of
+  // parameter pointers, most recently used first (at most kParamMapSets).
+  struct ParamMaps {
+    std::vector<const void*> ptrs;
+    std::unique_ptr<DevBlock> mem;
+  };
+  std::vector<ParamMaps> pmaps;
   // Device table of mirror destinations of the last X update, valid for the
   // host pointers in mirror_for (rebuilt when a call passes others).
   DevBlock mirror_mem;
@@ -344,6 +363,7 @@ struct Layout {
   size_t k1info = 0, k1items = 0, counters = 0, partials = 0, norms = 0;
   size_t k1tiles = 0;
   size_t total = 0;
+  std::vector<size_t> guards;
 };
 
 Layout plan_layout(const std::vector<Geom>& geom, bool with_ns, const TileLists* t) {
@@ -371,6 +391,7 @@ Layout plan_layout(const std::vector<Geom>& geom, bool with_ns, const TileLists*
   L.partials = a.take(sizeof(double) * L.k1tiles);
   L.norms = a.take(sizeof(double) * n);
   L.total = a.off;
+  L.guards = a.guards;
   return L;
 }
 
@@ -426,6 +447,9 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, long long k1_slack,
   }
   P->mem.bytes = lay.total;
   char* base = P->mem.ptr;
+  P->guards = lay.guards;
+  for (size_t g : lay.guards)
+    if (cudaMemset(base + g, kGuardByte, kGuardBytes) != cudaSuccess) return MUON_ERR_CUDA;
   long long xel = 0, ael = 0;
   P->x_off.resize(n);
   P->a_off.resize(n);
@@ -523,6 +547,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, long long k1_slack,
   P->k1.counters = reinterpret_cast<int*>(base + lay.counters);
   P->k1.partials = reinterpret_cast<double*>(base + lay.partials);
   P->k1.norms = reinterpret_cast<double*>(base + lay.norms);
+  P->k1.npartials = (int)lay.k1tiles;
   if (cudaMemcpy(P->k1.info, info.data(), sizeof(K1Info) * n, cudaMemcpyHostToDevice) != cudaSuccess)
     return MUON_ERR_CUDA;
   if (cudaMemcpy(P->k1.items, items.data(), sizeof(K1Item) * items.size(), cudaMemcpyHostToDevice) !=
@@ -589,6 +614,8 @@ int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, in
   L.info = P->k1.info;
   L.items = P->k1.items;
   L.nitems = P->k1.nitems;
+  L.n = n;
+  L.npartials = P->k1.npartials;
   L.mode = mode;
   L.nesterov = nesterov;
   L.beta = beta;
@@ -610,6 +637,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
            const FinalTable* F, cudaStream_t stream, const CUtensorMap* pmaps = nullptr,
            float* const* mirrors = nullptr, int n_mirrors = 0) {
   NsLaunch L;
+  L.nprobs = (int)P->geom.size();
   L.pmaps = nullptr;
   L.mirrors = nullptr;
   L.n_mirrors = 0;
@@ -682,37 +710,51 @@ std::vector<long long> shape_key(char kind, const std::vector<Geom>& geom) {
 }
 
 // Tensor maps over the caller's parameters for the TMA path of the last X
-// update.  They depend on the pointers, so they are rebuilt (after the stream
-// has drained, since queued kernels may still read the old ones) whenever a
-// call passes other pointers than the previous one.  Shapes whose row pitch
-// is not a multiple of 16 bytes use the register path (*out = nullptr).
+// update.  They depend on the pointers, so each plan keeps the maps of the
+// last kParamMapSets pointer sets, each in its own device block that is
+// written once, before any kernel reads it, and never changed while cached:
+// a call with a cached pointer set (a training loop alternating a few models
+// or parameter copies of one shape set) reuses its block and does not
+// synchronise.  Only when a new set evicts the least recently used block is
+// the stream synchronised first, since kernels queued earlier may still read
+// that block.  Shapes whose row pitch is not a multiple of 16 bytes use the
+// register path (*out = nullptr).
+constexpr size_t kParamMapSets = 8;
+
 int ensure_param_maps(Plan* P, float* const* params, int n, cudaStream_t stream,
                       const CUtensorMap** out) {
   *out = nullptr;
   for (int i = 0; i < n; ++i)
     if (P->geom[i].c % 4 != 0) return MUON_OK;
   std::vector<const void*> want(params, params + n);
-  if (P->pmap_mem.ptr && P->pmap_for == want) {
-    *out = reinterpret_cast<const CUtensorMap*>(P->pmap_mem.ptr);
+  for (size_t k = 0; k < P->pmaps.size(); ++k) {
+    if (P->pmaps[k].ptrs != want) continue;
+    if (k != 0) std::rotate(P->pmaps.begin(), P->pmaps.begin() + k, P->pmaps.begin() + k + 1);
+    *out = reinterpret_cast<const CUtensorMap*>(P->pmaps[0].mem->ptr);
     return MUON_OK;
-  }
-  if (!P->pmap_mem.ptr) {
-    if (cudaMalloc(&P->pmap_mem.ptr, sizeof(CUtensorMap) * n) != cudaSuccess) {
-      cudaGetLastError();
-      return MUON_ERR_NOMEM;
-    }
-    P->pmap_mem.bytes = sizeof(CUtensorMap) * n;
-  } else if (cudaStreamSynchronize(stream) != cudaSuccess) {
-    return MUON_ERR_CUDA;
   }
   std::vector<CUtensorMap> maps(n);
   for (int i = 0; i < n; ++i)
     if (!make_param_map(&maps[i], params[i], P->geom[i].r, P->geom[i].c)) return MUON_ERR_CUDA;
-  if (cudaMemcpy(P->pmap_mem.ptr, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice) !=
+  std::unique_ptr<DevBlock> blk;
+  if (P->pmaps.size() >= kParamMapSets) {
+    // The least recently used block may still be read by queued kernels.
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MUON_ERR_CUDA;
+    blk = std::move(P->pmaps.back().mem);
+    P->pmaps.pop_back();
+  } else {
+    blk.reset(new DevBlock());
+    if (cudaMalloc(&blk->ptr, sizeof(CUtensorMap) * n) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_NOMEM;
+    }
+    blk->bytes = sizeof(CUtensorMap) * n;
+  }
+  if (cudaMemcpy(blk->ptr, maps.data(), sizeof(CUtensorMap) * n, cudaMemcpyHostToDevice) !=
       cudaSuccess)
     return MUON_ERR_CUDA;
-  P->pmap_for = want;
-  *out = reinterpret_cast<const CUtensorMap*>(P->pmap_mem.ptr);
+  P->pmaps.insert(P->pmaps.begin(), Plan::ParamMaps{want, std::move(blk)});
+  *out = reinterpret_cast<const CUtensorMap*>(P->pmaps[0].mem->ptr);
   return MUON_OK;
 }
 
@@ -786,6 +828,12 @@ int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, 
 }
 
 }  // namespace
+
+unsigned long long current_wait_limit_ns() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return limit_ns();
+}
+
 }  // namespace muon
 
 using namespace muon;
@@ -1050,6 +1098,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
     ctx->stage_plans[key] = std::move(np);
   }
   NsLaunch L;
+  L.nprobs = 1;
   L.pmaps = nullptr;
   L.mirrors = nullptr;
   L.n_mirrors = 0;
@@ -1142,6 +1191,25 @@ int64_t muon_workspace_bytes(const int64_t* shapes, int n) {
   return tot;
 }
 
+int64_t muon_guard_check(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
+  int64_t changed = 0;
+  unsigned char h[kGuardBytes];
+  for (auto& kv : ctx->plans) {
+    const Plan& P = *kv.second;
+    for (size_t g : P.guards) {
+      if (cudaMemcpy(h, P.mem.ptr + g, kGuardBytes, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MUON_ERR_CUDA;
+      for (size_t b = 0; b < kGuardBytes; ++b) changed += (h[b] != kGuardByte);
+    }
+  }
+  return changed;
+}
+
 void muon_profile_begin(void) {
   std::lock_guard<std::mutex> lock(g_mutex);
   g_prof.on = true;
@@ -1186,6 +1254,31 @@ void muon_release(void) {
   cudaSetDevice(cur);
 }
 
-const char* muon_version(void) { return "muon-b200 0.1 (sm_100a, tcgen05)"; }
+const char* muon_version(void) {
+  return kBoundsCheck ? "muon-b200 0.2 (sm_100a, tcgen05, bounds-checked)"
+                      : "muon-b200 0.2 (sm_100a, tcgen05)";
+}
+
+#ifdef MUON_BOUNDS_CHECK
+int muon_debug_set_tile_row(const int64_t* shapes, int n, int index, int i0) {
+  if (check_shapes(shapes, n) || n < 1 || n > MUON_MAX_GROUP) return MUON_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCtx* ctx = nullptr;
+  int rc = get_ctx(&ctx);
+  if (rc) return rc;
+  auto it = ctx->plans.find(shape_key('S', make_geom(shapes, n)));
+  if (it == ctx->plans.end()) return MUON_ERR_INVALID_ARG;
+  NsPhase& ph = it->second->poly;
+  if (index < 0 || index >= ph.ntiles) return MUON_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
+  NsTile t;
+  if (cudaMemcpy(&t, ph.tiles + index, sizeof(t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  t.i0 = i0;
+  if (cudaMemcpy(ph.tiles + index, &t, sizeof(t), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+#endif
 
 }  // extern "C"

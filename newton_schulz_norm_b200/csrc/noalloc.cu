@@ -25,7 +25,6 @@
 // ordering) race on the array; order them on one stream.
 #include <algorithm>
 #include <cmath>
-#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -129,11 +128,6 @@ int g_blocks_per_sm[kMaxDevices] = {};
 
 long long cdiv_ll(long long a, long long b) { return (a + b - 1) / b; }
 
-unsigned long long noalloc_limit_ns() {
-  const char* s = std::getenv("MUON_SPIN_LIMIT_NS");
-  return (s && *s) ? std::strtoull(s, nullptr, 10) : 2000000000ull;
-}
-
 // Once per device: check the architecture and take the array's device address.
 int noalloc_device_setup(int dev, NoAllocScratch** scr, int* sms, int* bps) {
   if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
@@ -195,6 +189,7 @@ extern "C" int muon_momentum_normalize_noalloc(const float* const* grads, float*
   }
   S.n = n;
   S.nitems = (int)(2 * items);
+  const unsigned long long limit = current_wait_limit_ns();   // before this file's own lock
 
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   int dev = 0;
@@ -214,6 +209,8 @@ extern "C" int muon_momentum_normalize_noalloc(const float* const* grads, float*
   L.info = scr->info;
   L.items = scr->items;
   L.nitems = S.nitems;
+  L.n = n;
+  L.npartials = kMaxItems / 2;
   L.mode = K1_MOMENTUM;
   L.nesterov = nesterov;
   L.beta = beta;
@@ -222,7 +219,7 @@ extern "C" int muon_momentum_normalize_noalloc(const float* const* grads, float*
   L.ready = scr->counters + 1 + n;
   L.partials = scr->partials;
   L.norms = scr->norms;
-  L.limit_ns = noalloc_limit_ns();
+  L.limit_ns = limit;
   L.status = dev_status ? dev_status : &scr->status;
   for (int i = 0; i < n; ++i) {
     L.ptrs[i].g = grads[i];

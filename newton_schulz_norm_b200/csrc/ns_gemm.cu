@@ -378,7 +378,28 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
   const uint32_t tmem = *tmem_slot;
   const unsigned long long limit = L.limit_ns;
 
-  if (warp == 0) {
+  // Checked builds: both CTAs of the pair validate every tile the pair owns
+  // (the same list, so they agree) and refuse all of them if one is invalid.
+  bool refuse = false;
+  if (kBoundsCheck) {
+    int bad = 0;
+    for (int t = pair + (int)threadIdx.x * npairs; t < L.ntiles; t += (int)blockDim.x * npairs) {
+      const NsTile tl = L.tiles[t];
+      bool ok = tl.prob >= 0 && tl.prob < L.nprobs;
+      if (ok) {
+        const NsProblem& Q = L.probs[tl.prob];
+        ok = tl.i0 >= 0 && tl.i0 < Q.M && tl.j0 >= 0 && tl.j0 < Q.N && tl.kc > 0 &&
+             (long long)tl.kc * BK >= Q.K && Q.slot >= 0 && Q.slot < MUON_MAX_GROUP;
+      }
+      bad |= ok ? 0 : 1;
+    }
+    refuse = __syncthreads_or(bad) != 0;
+    if (refuse && threadIdx.x == 0) record_status(L.status, MUON_ERR_INVALID_ARG);
+  }
+
+  if (refuse) {
+    // nothing issued: straight to the teardown
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;

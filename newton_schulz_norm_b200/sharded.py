@@ -139,8 +139,23 @@ class ShardedMuon:
 
     def step(self, grads: Sequence[torch.Tensor], lr: float, beta: float = 0.95,
              nesterov: bool = True, coeffs=None, stream=None) -> None:
+        """One step.  ``stream`` (default: torch's current stream) runs the
+        owned matrices' kernels, after everything already queued on torch's
+        current stream (the previous step's exchange included).  The
+        exchange (all-gather, or the device barrier of the fused mode) runs
+        on torch's current stream, which is made to wait for ``stream``
+        first, so it never reads parameters the kernels have not written
+        yet.  In the fused mode every rank's kernels also wait for a device
+        barrier at entry: no rank stores into another rank's copy while that
+        rank may still be reading its parameters from before this step."""
         if len(grads) != len(self.shapes):
             raise ValueError("one gradient per matrix is required")
+        cur = torch.cuda.current_stream() if self.flat.is_cuda else None
+        side = stream is not None and cur is not None and stream != cur
+        if self.fused:
+            self._symm.barrier()     # every rank is done with its parameters of the last step
+        if side:
+            stream.wait_stream(cur)  # after the entry barrier and the last step's exchange
         if self.owned:
             kw = dict(lr=lr, beta=beta, nesterov=nesterov, ns_steps=self.ns_steps)
             if coeffs is not None:
@@ -151,6 +166,8 @@ class ShardedMuon:
                 kw["mirrors"] = self._mirrors
             self.step_fn([self.params[i] for i in self.owned], [grads[i] for i in self.owned],
                          [self.bufs[i] for i in self.owned], **kw)
+        if side:
+            cur.wait_stream(stream)  # the exchange below runs after the kernels
         if self.fused:
             self._symm.barrier()     # every rank's peer stores are done and visible
         else:

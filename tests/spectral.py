@@ -65,3 +65,26 @@ def lift_threshold(target=0.6, coeffs=DEFAULT_COEFFS, steps=5):
         else:
             lo = mid
     return hi
+
+
+def band_report(x_out, u, coeffs=DEFAULT_COEFFS, steps=5, low=0.6, high=1.3, slack=0.02):
+    """The singular-value band of one orthogonalised update, read as stated
+    for the literal [0.6, 1.3] band (which low-rank gradients cannot meet):
+
+    * every singular value of the output is at most ``high``;
+    * at least as many output singular values reach ``low - slack`` as the
+      normalised input u/||u|| has singular values at or above the lift
+      threshold (the smallest s0 that ``steps`` iterations of p carry to
+      ``low``): every direction the iteration can lift is lifted.
+
+    Returns (max_sigma, lifted_out, liftable_in, literal_fraction), the last
+    being the fraction of output singular values inside [low, high]."""
+    x = np.asarray(x_out, dtype=np.float64)
+    sv = np.linalg.svd(x, compute_uv=False)
+    u = np.asarray(u, dtype=np.float64)
+    s0 = np.linalg.svd(u / np.linalg.norm(u), compute_uv=False)
+    thr = lift_threshold(low, coeffs, steps)
+    lifted = int(np.sum(sv >= low - slack))
+    liftable = int(np.sum(s0 >= thr))
+    literal = float(np.mean((sv >= low) & (sv <= high))) if sv.size else 1.0
+    return float(sv.max()) if sv.size else 0.0, lifted, liftable, literal

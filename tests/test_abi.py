@@ -38,6 +38,20 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, s), s
 
 
+def test_checked_build_exports_debug_symbols():
+    """The bounds-checked variant exports every muon.h symbol and the
+    muon_debug.h ones; the regular library does not export the latter."""
+    from newton_schulz_norm_b200 import build
+    import newton_schulz_norm_b200 as m
+    chk = ctypes.CDLL(build.build(checked=True))
+    text = open(os.path.join(ROOT, "include", "muon_debug.h")).read()
+    dbg = sorted(set(re.findall(r"MUON_API\s+[\w\s\*]*?\b(muon_\w+)\s*\(", text)))
+    assert dbg == ["muon_debug_set_tile_row"]
+    for s in _declared_symbols() + dbg:
+        assert hasattr(chk, s), s
+    assert not hasattr(m.library(), dbg[0])
+
+
 def test_no_cpu_fallback_symbols(lib):
     # The library is CUDA-only: its entry points are the declared ones, and the
     # package carries no oracle import.

@@ -12,18 +12,22 @@ Tolerances (from the arithmetic, stated per check):
   matters only for entries that cancel to near zero), and differ on at most
   1% of entries.
 * orthogonalised update (Delta p = -lr*s*X5) and new parameters: relative
-  Frobenius error <= 1e-2 for a single orthogonalisation and for a step from
-  zero momentum (measured <= 0.82%).  The bf16 iteration is chaotic:
-  directions with small singular values grow up to a = 3.44-fold per
-  iteration, so the rare accumulation-order roundings above grow with every
-  iteration (0.01%, 0.05%, 0.25%, 0.5%, 0.8% after 1..5 iterations).  The
-  tensor core accumulates in fp32 truncated toward zero; a CPU model of the
-  same algorithm with that accumulation (exact sums of 16 products, then an
-  fp32 accumulator truncated toward zero) lands as far from the oracle as
-  the GPU does (0.81% / 0.70% vs 0.78% / 0.66% at step 1, 0.99% / 0.87% vs
-  0.95% / 0.86% at step 2), while round-to-nearest fp32 would land at 0.4%.
-  Along a momentum trajectory the spectrum of u hardens and both reach
-  ~1.3% by step 8; those cases are held to X_TOL_TRAJ = 1.5e-2.
+  Frobenius error <= 1e-2 (X_TOL) for a single orthogonalisation and for a
+  step from zero momentum (measured <= 0.82%).
+* steps taken after momentum has accumulated (every GPT-2 124M, medium and XL
+  step, steps 2-10 of the GPT-2 block): <= 1.5e-2 (X_TOL_TRAJ), because
+  1e-2 is out of reach of the tensor core's arithmetic, not of the kernels.
+  The bf16 iteration is chaotic: directions with small singular values grow
+  up to a = 3.44-fold per iteration, so any difference in an accumulation
+  that flips a bf16 rounding grows with every iteration.  The tensor core
+  adds each exact 16-product sum into an fp32 accumulator truncated toward
+  zero; tests/tc_model.py models that, and its distance from the oracle
+  matches the GPU's step by step (checked below, on the GPU, on every step
+  of the GPT-2 block trajectory).  At step 8 of that trajectory (768 x 2304)
+  the model lands 1.34% from the oracle (the GPU 1.30%); split-K
+  accumulation over four partial accumulators would still land 1.18% away,
+  and round-to-nearest fp32 accumulation, which this hardware does not offer,
+  1.05% (tests/test_tc_model.py pins both of the latter above 1e-2).
 """
 import math
 
@@ -35,7 +39,8 @@ from oracle import (coeffs_f32, momentum_ref, muon_step_ref, newton_schulz_ref, 
                     orient, orthogonalize_ref)
 from tests.gpu_util import (bf16_agreement, bf16_close, fp32_gemm_bound, rel_fro, to_bf16, to_f32,
                             to_np)
-from tests.spectral import lift_threshold, poly_scalar
+from tests.spectral import band_report, lift_threshold, poly_scalar
+from tests.tc_model import orthogonalize_tc
 from workloads import WORKLOADS, WorkloadStream, square_case
 
 pytestmark = pytest.mark.gpu
@@ -205,9 +210,15 @@ def test_square_sweep_vs_oracle(muon, n):
     assert np.linalg.norm(off) / np.linalg.norm(target) < 5e-2
 
 
-def test_square_4096_closed_form(muon):
+def test_square_4096_vs_oracle(muon):
+    """The 4096 square of the sweep (randomised-Hadamard factors) against the
+    oracle at the 1e-2 bar, and through its known factors."""
     case = square_case(4096, seed=0)
     out = to_np(muon.orthogonalize(to_f32(case.g), ns_steps=5))
+    ref = orthogonalize_ref(case.g, 5, COEFFS)
+    err = rel_fro(out, ref)
+    print(f"n = 4096: GPU vs oracle {err:.4%}")
+    assert err <= X_TOL
     d = case.project(out)
     target = poly_scalar(case.sigma / np.linalg.norm(case.sigma), COEFFS, 5)
     assert rel_fro(np.diag(d), target) < 3e-2
@@ -242,6 +253,24 @@ def _check_step(p_old, p_gpu, b_gpu, p_ref, b_ref, tol=X_TOL):
         assert errs[-1][1] <= tol, errs[-1]
     if den > 0:
         assert math.sqrt(num / den) <= tol, errs
+
+
+def _step_x(p_old, p_new, lr):
+    """The orthogonalised update X5 a step applied, recovered from the
+    parameters: p_new = fp32(p_old - s X5), s = fp32(lr sqrt(max(1, r/c)))."""
+    r, c = p_old.shape
+    s = float(np.float32(float(np.float32(lr)) * math.sqrt(max(1.0, r / c))))
+    new = to_np(p_new) if isinstance(p_new, torch.Tensor) else np.asarray(p_new, np.float64)
+    return (np.asarray(p_old, np.float64) - new) / s
+
+
+def _check_band(x5, u, what):
+    """The singular-value band of one step's update (see tests/spectral.py):
+    max sigma <= 1.3 and every liftable direction lifted to >= 0.6 (- 0.02)."""
+    smax, lifted, liftable, literal = band_report(x5, u)
+    assert smax <= 1.3, (what, smax)
+    assert lifted >= liftable, (what, lifted, liftable)
+    return literal
 
 
 EDGE_SHAPES = [(1, 1), (1, 100), (100, 1), (7, 13), (13, 7), (64, 64), (129, 257), (257, 129),
@@ -288,8 +317,18 @@ def test_step_zero_grad_and_nan_isolation(muon):
     _check_step(ps[2:], p_d[2:], b_d[2:], p_ref, b_ref)
 
 
-@pytest.mark.parametrize("name,steps", [("single_256", 3), ("gpt2_block", 3)])
-def test_step_workloads_consecutive(muon, name, steps):
+@pytest.mark.parametrize("name", ["single_256", "gpt2_block"])
+def test_step_workloads_consecutive(muon, name):
+    """Every step the workload specifies (3 for the single matrix, 10 for the
+    GPT-2 block), each compared with the oracle from identical inputs: the two
+    trajectories are put back on the oracle's state after every step.  Every
+    step's update also passes the singular-value band.
+
+    For the GPT-2 block, every step of the 768 x 768 matrix (attn c_proj) is
+    also compared with the tensor-core accumulation model (tests/tc_model.py)
+    on the same input: the GPU must land as far from the oracle as the model
+    of its truncating fp32 accumulation predicts (within 15% + 0.1%), which
+    is what carries these steps past the 1e-2 bar (module docstring)."""
     wl = WORKLOADS[name]
     st = WorkloadStream(wl, seed=0)
     params, bufs = st.init()
@@ -297,9 +336,11 @@ def test_step_workloads_consecutive(muon, name, steps):
     b_d = [to_f32(b) for b in bufs]
     p_ref = [p.copy() for p in params]
     b_ref = [b.copy() for b in bufs]
-    for k in range(steps):
+    model_rows = []
+    for k in range(wl.steps):
         grads = st.next_grads()
         p_old = [p.copy() for p in p_ref]
+        b_old = [b.copy() for b in b_ref]
         muon.step(p_d, [to_f32(g) for g in grads], b_d, lr=wl.lr, beta=wl.beta,
                   nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
         torch.cuda.synchronize()
@@ -307,35 +348,54 @@ def test_step_workloads_consecutive(muon, name, steps):
                                      nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
         zero_momentum = k == 0 and wl.buf_std == 0
         _check_step(p_old, p_d, b_d, p_ref, b_ref, tol=X_TOL if zero_momentum else X_TOL_TRAJ)
+        for i in range(len(p_d)):
+            _, u = momentum_ref(grads[i], b_old[i], wl.beta, wl.nesterov)
+            _check_band(_step_x(p_old[i], p_d[i], wl.lr), u, (name, k, i))
+        if name == "gpt2_block":
+            i = 1
+            _, u = momentum_ref(grads[i], b_old[i], wl.beta, wl.nesterov)
+            x_ref = orthogonalize_ref(u, wl.ns_steps, wl.coeffs)
+            e_gpu = rel_fro(_step_x(p_old[i], p_d[i], wl.lr), x_ref)
+            e_model = rel_fro(orthogonalize_tc(u, wl.ns_steps, wl.coeffs), x_ref)
+            model_rows.append((k + 1, e_gpu, e_model))
         # keep the two trajectories on the same state, so that each step is
         # compared from identical inputs
         for i in range(len(p_d)):
             p_d[i].copy_(to_f32(p_ref[i]))
             b_d[i].copy_(to_f32(b_ref[i]))
+    for k, e_gpu, e_model in model_rows:
+        print(f"step {k}: GPU vs oracle {e_gpu:.4%}, tensor-core model vs oracle {e_model:.4%}")
+        assert abs(e_gpu - e_model) <= 0.15 * e_model + 1e-3, (k, e_gpu, e_model)
     assert muon.status() == 0
 
 
-def test_step_gpt2_124m_full_size_sampled(muon):
-    """All 48 matrices in one call (the benchmarked launch configuration);
-    the oracle recomputes a sample of them (one of each shape and the last)."""
+def test_step_gpt2_124m_all_48_first_3_steps(muon):
+    """All 48 matrices in one call (the benchmarked launch configuration),
+    the first three steps of the workload, every matrix against the oracle
+    (momentum is warm-started, so every step is a trajectory step); one
+    matrix of each shape per step passes the singular-value band."""
     wl = WORKLOADS["gpt2_124m"]
     st = WorkloadStream(wl, seed=0)
     params, bufs = st.init()
-    grads = st.next_grads()
-    p_d, b_d = _run_step(muon, params, grads, bufs, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov,
-                         ns_steps=wl.ns_steps, coeffs=wl.coeffs)
-    assert muon.status() == 0
-    sample = [0, 1, 2, 3, 47]
-    p_ref, b_ref = muon_step_ref([params[i] for i in sample], [grads[i] for i in sample],
-                                 [bufs[i] for i in sample], lr=wl.lr, beta=wl.beta,
-                                 nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
-    # momentum is warm-started (N(0, 0.1^2)), so this is a trajectory step
-    _check_step([params[i] for i in sample], [p_d[i] for i in sample], [b_d[i] for i in sample],
-                p_ref, b_ref, tol=X_TOL_TRAJ)
-    # property at full size: every momentum buffer matches the one-rounding form
-    for i in range(0, 48, 7):
-        br, _ = momentum_ref(grads[i], bufs[i], wl.beta, wl.nesterov)
-        assert np.max(np.abs(to_np(b_d[i]) - br)) <= BUF_TOL * np.max(np.abs(br))
+    p_d = [to_f32(p) for p in params]
+    b_d = [to_f32(b) for b in bufs]
+    p_ref, b_ref = params, bufs
+    for k in range(3):
+        grads = st.next_grads()
+        p_old, b_old = p_ref, b_ref
+        muon.step(p_d, [to_f32(g) for g in grads], b_d, lr=wl.lr, beta=wl.beta,
+                  nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+        torch.cuda.synchronize()
+        assert muon.status() == 0
+        p_ref, b_ref = muon_step_ref(p_old, grads, b_old, lr=wl.lr, beta=wl.beta,
+                                     nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+        _check_step(p_old, p_d, b_d, p_ref, b_ref, tol=X_TOL_TRAJ)
+        for i in (0, 1, 2, 3):
+            _, u = momentum_ref(grads[i], b_old[i], wl.beta, wl.nesterov)
+            _check_band(_step_x(p_old[i], p_d[i], wl.lr), u, (k, i))
+        for i in range(48):
+            p_d[i].copy_(to_f32(p_ref[i]))
+            b_d[i].copy_(to_f32(b_ref[i]))
 
 
 def test_update_scale_on_transposed(muon):
@@ -386,33 +446,54 @@ def test_rejects_bad_args_before_launch(muon):
     assert torch.all(b == 0)
 
 
-def _first_step_sampled(muon, wl, subset_layers, sample):
-    """One step on the listed layers' matrices (all in one call), the oracle on
-    `sample` (indices into the call's matrices)."""
-    idx = [4 * l + k for l in subset_layers for k in range(4)]
-    st = WorkloadStream(wl, seed=0, subset=idx)
-    params, bufs = st.init()
-    grads = st.next_grads()
-    p_d, b_d = _run_step(muon, params, grads, bufs, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov,
-                         ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+def _first_step_sampled(muon, wl, sample, band=()):
+    """One step on every matrix of the workload in one call; the oracle on
+    the matrices in ``sample``.  Inputs are drawn matrix by matrix and moved
+    to the GPU at once, so the host keeps only the sampled ones."""
+    st = WorkloadStream(wl, seed=0)
+    keep = set(sample)
+    p_d, b_d, g_d, host = [], [], [], {}
+    for i, p, b in st.init_iter():
+        p_d.append(to_f32(p))
+        b_d.append(to_f32(b))
+        if i in keep:
+            host[i] = [p, b, None]
+    for i, g in st.grads_iter():
+        g_d.append(to_f32(g))
+        if i in keep:
+            host[i][2] = g
+    muon.step(p_d, g_d, b_d, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov,
+              ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    torch.cuda.synchronize()
     assert muon.status() == 0
-    p_ref, b_ref = muon_step_ref([params[i] for i in sample], [grads[i] for i in sample],
-                                 [bufs[i] for i in sample], lr=wl.lr, beta=wl.beta,
+    del g_d
+    params = [host[i][0] for i in sample]
+    bufs = [host[i][1] for i in sample]
+    grads = [host[i][2] for i in sample]
+    p_ref, b_ref = muon_step_ref(params, grads, bufs, lr=wl.lr, beta=wl.beta,
                                  nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
     # warm-started momentum: a trajectory step
-    _check_step([params[i] for i in sample], [p_d[i] for i in sample], [b_d[i] for i in sample],
-                p_ref, b_ref, tol=X_TOL_TRAJ)
+    _check_step(params, [p_d[i] for i in sample], [b_d[i] for i in sample], p_ref, b_ref,
+                tol=X_TOL_TRAJ)
+    for k, i in enumerate(sample):
+        if i in band:
+            _, u = momentum_ref(grads[k], bufs[k], wl.beta, wl.nesterov)
+            _check_band(_step_x(params[k], p_d[i], wl.lr), u, i)
 
 
 def test_step_gpt2_medium_all_96_sampled(muon):
-    """GPT-2 medium shapes (d = 1024): all 96 matrices in one call."""
-    _first_step_sampled(muon, WORKLOADS["gpt2_medium"], range(24), sample=[0, 1, 2, 3])
+    """GPT-2 medium shapes (d = 1024): all 96 matrices in one call; the
+    oracle on the first and the last layer."""
+    _first_step_sampled(muon, WORKLOADS["gpt2_medium"], sample=[0, 1, 2, 3, 92, 93, 94, 95],
+                        band=(0, 1, 2, 3))
 
 
-def test_step_gpt2_xl_two_layers_sampled(muon):
-    """GPT-2 XL shapes (d = 1600, not a multiple of the 256-wide tiles):
-    two layers (8 matrices) in one call, every shape checked."""
-    _first_step_sampled(muon, WORKLOADS["gpt2_xl"], [0, 47], sample=[0, 1, 2, 3, 7])
+def test_step_gpt2_xl_all_192_sampled(muon):
+    """GPT-2 XL shapes (d = 1600, not a multiple of the 256-wide tiles): all
+    192 matrices (1.47e9 elements) in one call, the largest workload; the
+    oracle on every shape of the first and the last layer."""
+    _first_step_sampled(muon, WORKLOADS["gpt2_xl"], sample=[0, 1, 2, 3, 188, 189, 190, 191],
+                        band=(1,))
 
 
 def test_square_8192_closed_form(muon):

@@ -55,8 +55,30 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     class A:
         steps, warmup, gpus = 1, 0, 2
-    assert bench.run_reference(A, WORKLOADS["gpt2_124m"], rank=1) == 0
+    assert bench.run_reference(A, WORKLOADS["gpt2_124m"], rank=1, world=2) == 0
     assert capsys.readouterr().out == ""           # no line, no work on rank 1
+
+
+def test_reference_arm_line_is_self_consistent(capsys):
+    """Rank 0's line: steps x ms_per_step is the time actually spent in the
+    timed oracle calls, value scales one call to the whole workload, and the
+    config is the one the GPU arm prints."""
+    import json
+    import bench
+    from workloads import WORKLOADS
+
+    class A:
+        steps, warmup, gpus = 2, 0, 1
+    wl = WORKLOADS["gpt2_124m"]
+    assert bench.run_reference(A, wl, rank=0, world=1) == 0
+    d = json.loads(capsys.readouterr().out.strip())
+    assert d["impl"] == "reference" and d["steps"] == 2
+    sc = d["sampled_calls"]
+    assert sc["calls"] == 2 and sc["matrices_per_call"] == 4
+    assert abs(d["steps"] * d["ms_per_step"] - 1e3 * sc["seconds_timed"]) < 1e-6 * d["ms_per_step"] + 1e-3
+    assert abs(d["value"] - d["ms_per_step"] * wl.n_matrices / 4) < 1e-9 * d["value"]
+    assert d["config"] == dict(bench.workload_config(wl), parallelism=bench.parallelism(1))
+    assert d["cpu_baseline"]["value"] == d["value"] and d["e2e"]["value"] == d["value"]
 
 
 def test_single_rank_needs_no_process_group():

@@ -15,6 +15,9 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import momentum_ref, normalize_ref, orient
+from workloads import WORKLOADS, WorkloadStream
+
 pytestmark = pytest.mark.gpu
 
 BUF_TOL = 1e-6
@@ -65,6 +68,43 @@ def test_noalloc_matches_allocating_entry_point_two_calls(muon):
             ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(a), 2.0 ** -126))) - 7)
             assert np.all(np.abs(a - b) <= ulp), (call, (r, c))
             assert np.mean(a != b) <= 1e-3, (call, (r, c))
+
+
+def test_noalloc_gpt2_124m_queue_order_and_oracle(muon):
+    """All 48 GPT-2 124M matrices: 5184 first-pass work items, far more than
+    the queue slack (half the resident CTAs), so the set-up kernel splits
+    first-pass runs to queue each matrix's second pass in between (the order
+    the allocating entry point builds on the host).  Two calls in a row must
+    match the allocating entry point and report no timeout; a sample of the
+    outputs is also checked against the oracle (one bf16 rounding of the same
+    fp32 u over its norm: within one bf16 ulp)."""
+    wl = WORKLOADS["gpt2_124m"]
+    st = WorkloadStream(wl, seed=5)
+    _, bufs0 = st.init()
+    b_ref = [torch.from_numpy(b).cuda() for b in bufs0]
+    b_na = [torch.from_numpy(b).cuda() for b in bufs0]
+    x_na = _x0_buffers(wl.shapes)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sample = [0, 3, 46]
+    for call in range(2):
+        grads_np = st.next_grads()
+        grads = [torch.from_numpy(g).cuda() for g in grads_np]
+        b_before = [bufs0[i] if call == 0 else b_na[i].cpu().numpy() for i in sample]
+        x_ref = muon.momentum_normalize(grads, b_ref, beta=wl.beta, nesterov=wl.nesterov)
+        code = muon.momentum_normalize_noalloc(grads, b_na, x_na, beta=wl.beta,
+                                               nesterov=wl.nesterov, dev_status=status)
+        assert code == 0
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for (r, c), br, bn, xr, xn in zip(wl.shapes, b_ref, b_na, x_ref, x_na):
+            assert torch.equal(br, bn), (call, (r, c))
+            assert torch.equal(xr, xn[:, :max(r, c)]), (call, (r, c))
+        for k, i in enumerate(sample):
+            _, u = momentum_ref(grads_np[i], b_before[k], wl.beta, wl.nesterov)
+            want, _ = orient(normalize_ref(u))
+            got = x_na[i][:, :want.shape[1]].float().cpu().numpy().astype(np.float64)
+            ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(want), 2.0 ** -126))) - 7)
+            assert np.all(np.abs(got - want) <= ulp), (call, i)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(muon):

@@ -134,39 +134,52 @@ class WorkloadStream:
     def _want(self, i: int) -> bool:
         return self.subset is None or i in self.subset
 
-    def init(self) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+    def init_iter(self):
+        """Yield (i, p, buf) for every matrix in listing order (the subset is
+        ignored), so that a caller can move each matrix elsewhere before the
+        next is drawn.  Draws exactly what ``init()`` draws."""
         assert not self._initialised
         self._initialised = True
-        params, bufs = [], []
         for i, (r, c) in enumerate(self.wl.shapes):
             p = _normal32(self.rng, (r, c), self.wl.param_std)
             if self.wl.buf_std > 0:
                 b = _normal32(self.rng, (r, c), self.wl.buf_std)
             else:
                 b = np.zeros((r, c), np.float32)
+            yield i, p, b
+
+    def init(self) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+        params, bufs = [], []
+        for i, p, b in self.init_iter():
             if self._want(i):
                 params.append(p)
                 bufs.append(b)
         return params, bufs
 
-    def next_grads(self) -> List[np.ndarray]:
-        out = []
+    def grads_iter(self, want=None):
+        """Yield (i, g) for the next step's gradient of every matrix i with
+        ``want(i)`` true (default: every matrix), drawing the random stream of
+        all of them in listing order.  Draws exactly what ``next_grads()``
+        draws."""
         k = self.wl.grad_rank
         for i, (r, c) in enumerate(self.wl.shapes):
+            keep = want is None or want(i)
             if k == 0:
                 g = _normal32(self.rng, (r, c))
             else:
                 A = _normal32(self.rng, (r, k))
                 B = _normal32(self.rng, (c, k))
                 noise = _normal32(self.rng, (r, c), self.wl.grad_noise)
-                if not self._want(i):
+                if not keep:
                     continue
                 # fp64 product then one rounding: independent of BLAS blocking.
                 g = (A.astype(np.float64) @ B.astype(np.float64).T).astype(np.float32)
                 g += noise
-            if self._want(i):
-                out.append(g)
-        return out
+            if keep:
+                yield i, g
+
+    def next_grads(self) -> List[np.ndarray]:
+        return [g for _, g in self.grads_iter(self._want)]
 
 
 def haar_orthogonal(rng: np.random.Generator, n: int) -> np.ndarray:
