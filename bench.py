@@ -53,12 +53,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import ADAMW_WORKLOADS, WORKLOADS, AdamWStream, WorkloadStream  # noqa: E402
+from workloads import (ADAMW_WORKLOADS, SQUARE_SWEEP, WORKLOADS, AdamWStream,  # noqa: E402
+                       WorkloadStream, square_case)
 
 METRIC = "Muon step ms, GPT-2 124M 48 mats; Newton-Schulz bf16 TFLOP/s vs tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 N_GRAD_SETS = 4
-KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply")
+KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "ns_chain")
 ADAMW_BYTES_PER_ELEMENT = 28.0     # read p, g, m, v; write p, m, v (fp32)
 
 
@@ -68,7 +69,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="gpt2_124m", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="gpt2_124m",
+                    choices=sorted(WORKLOADS) + [f"square_{n}" for n in SQUARE_SWEEP])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW side measurement")
@@ -121,6 +123,7 @@ def per_launch_work(wl):
         p += m ** 3             # symmetric square
         u += 2 * m * m * n      # X update
     el = wl.n_elements
+    k = wl.ns_steps
     return {
         "momentum_norm_cast": ("hbm", 14.0 * el),     # read g, buf; write buf (fp32); write X0 (bf16)
         "gram": ("tensor", g),
@@ -128,6 +131,8 @@ def per_launch_work(wl):
         "xupdate": ("tensor", u),
         "xupdate_final": ("tensor", u),
         "apply": ("hbm", 10.0 * el),
+        # one launch: every Gram, polynomial and X-update phase but the last update
+        "ns_chain": ("tensor", (g + p) * k + u * max(0, k - 1)),
     }
 
 
@@ -135,7 +140,7 @@ def per_launch_work(wl):
 KIND_SOURCES = {
     "momentum_norm_cast": ("momentum.cu",),
     "gram": ("ns_gemm.cu",), "poly": ("ns_gemm.cu",), "xupdate": ("ns_gemm.cu",),
-    "xupdate_final": ("ns_gemm.cu",), "apply": ("momentum.cu",),
+    "xupdate_final": ("ns_gemm.cu",), "apply": ("momentum.cu",), "ns_chain": ("ns_gemm.cu",),
     "adamw": ("adamw.cu",),
 }
 _SHARED_SOURCES = ("internal.h", "ptx.cuh", "muon_api.cu")
@@ -742,7 +747,7 @@ def run_ours(args, wl, rank, world):
     tot_all = sum(prof[k][0] for k in KINDS)
     for k in kernels:
         kernels[k]["share"] = prof[k][0] / tot_all
-    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "xupdate", "xupdate_final")) / args.steps
+    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "xupdate", "xupdate_final", "ns_chain")) / args.steps
     ns_tflops = wl.ns_flops() / (ns_ms * 1e-3) / 1e12
     launches = sum(prof[k][1] for k in KINDS)
 
@@ -775,10 +780,117 @@ def run_ours(args, wl, rank, world):
     return 0
 
 
+def run_square(args, n, rank, world):
+    """The square sweep: one Newton-Schulz orthogonalisation (muon_orthogonalize,
+    5 quintic steps, bf16) of an n x n matrix U diag(sigma) V^T with log-uniform
+    sigma (condition number 1e3) per step; fp32 in, bf16 out.  Rank r of N
+    orthogonalises its own matrix (seed = rank): weak scaling."""
+    import torch
+    import newton_schulz_norm_b200 as muon
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks(world, "nccl", dev)
+    case = square_case(n, seed=rank_seed(rank))
+    flops = 20.0 * n ** 3                     # (3 m^2 n + m^3) x 5 with m = n
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import orthogonalize_ref
+        m = min(n, 4096)                      # the oracle on the same matrix size up to 4096
+        sub = square_case(m, seed=0)
+        t0 = time.perf_counter()
+        orthogonalize_ref(sub.g, 5, (3.4445, -4.7750, 2.0315))
+        secs = time.perf_counter() - t0
+        scale = (n / m) ** 3
+        cpu_base = {"value": 1e3 * secs * scale, "unit": "ms", "cores": blas_threads(),
+                    "kind": "oracle",
+                    "sample": f"oracle on one {m} x {m} orthogonalisation, {secs:.1f} s"
+                              + (f", scaled x{scale:g} (n^3)" if scale != 1 else "")}
+    x = torch.from_numpy(case.g).to(dev)
+    out = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        muon.orthogonalize(x, out=out)
+    torch.cuda.synchronize()
+    muon.profile_begin()
+    for _ in range(args.steps):
+        muon.orthogonalize(x, out=out)
+    torch.cuda.synchronize()
+    prof = muon.profile_end()
+    time.sleep(0.25)
+    ranks.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        muon.orthogonalize(x, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(e0.elapsed_time(e1) / args.steps)
+    if muon.status() != 0:
+        raise RuntimeError("device-side error")
+    # e2e: fp32 matrix in from pinned host memory, bf16 result out, every step
+    hx = torch.from_numpy(case.g).pin_memory()
+    hout = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
+    torch.cuda.synchronize()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        x.copy_(hx, non_blocking=True)
+        muon.orthogonalize(x, out=out)
+        hout.copy_(out, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ranks.max(e2.elapsed_time(e3) / args.steps)
+    peaks = load_peaks()
+    chain_ms, chain_n = prof["ns_chain"]
+    fin_ms, fin_n = prof["xupdate_final"]
+    chain_flops = flops - 2.0 * n ** 3        # every phase but the last update
+    ach = chain_flops / (chain_ms / chain_n * 1e-3) / 1e12
+    kernels = {k: {"launches": v[1], "ms_per_launch": v[0] / v[1]} for k, v in prof.items() if v[1]}
+    out_line = {
+        "metric": f"Newton-Schulz orthogonalisation ms, {n}x{n}; bf16 TFLOP/s vs tensor peak",
+        "value": ms, "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"square_{n}: one {n} x {n} fp32 matrix U diag(sigma) V^T, sigma "
+                               f"log-uniform on [1e-3, 1], 5 NS steps, coeffs [3.4445, -4.775, 2.0315], "
+                               f"bf16 output", "parallelism": parallelism(world),
+                   "ns_flop_per_step": flops,
+                   "l2": f"input {4 * n * n / 1e6:.0f} MB fp32, iterates {2 * 2 * n * n / 1e6:.0f} MB bf16"},
+        "tflops": flops / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "ns_chain", "achieved": ach,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peaks['source']} (burst)", "work_per_launch": chain_flops,
+                     "avg_launch_ms": chain_ms / chain_n},
+        "kernels": kernels,
+        "cpu_baseline": cpu_base,
+        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * n * n,
+                "d2h_bytes_per_step": 2 * n * n},
+        "gpu_launches": sum(v[1] for v in prof.values()) // max(1, args.steps) * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(out_line), flush=True)
+    ranks.close()
+    return 0
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.workload.startswith("square_"):
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the square sweep's oracle "
+                                  "time is reported in the GPU line's cpu_baseline"}))
+            return 0
+        return run_square(args, int(args.workload.split("_")[1]), rank, world)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl, rank, world)

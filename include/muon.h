@@ -270,10 +270,13 @@ MUON_API int64_t muon_workspace_bytes(const int64_t* shapes, int n);
  *   0 momentum/norm/cast   1 Gram   2 polynomial   3 X update
  *   4 X update with the fused parameter update   5 update without NS steps
  *   6 AdamW (muon_adamw_step)
+ *   7 the chain launch: every Gram, polynomial and X-update phase of a step
+ *     but the last update (kinds 1-3 are then used only by the stage entry
+ *     points)
  * ms and launches are host arrays of at least nkinds entries.  Returns the
  * number of kinds written, or a negative status.
  */
-#define MUON_PROFILE_KINDS 7
+#define MUON_PROFILE_KINDS 8
 MUON_API void muon_profile_begin(void);
 MUON_API int muon_profile_end(double* ms, int64_t* launches, int nkinds);
 

@@ -23,13 +23,13 @@ extern "C" {
 
 /*
  * muon_debug_set_tile_row -- overwrite the first output row (i0) of tile
- * `index` of the polynomial phase of the plan cached for this shape set (the
- * plan a muon_step call with these shapes built), so that the next muon_step
- * on these shapes meets an invalid tile.  Synchronises the device.  Returns
- * MUON_OK, MUON_ERR_INVALID_ARG if no such plan or tile exists.  The plan
- * stays corrupted until muon_release().
+ * `index` of the chain launch of `ns_steps` iterations cached for this shape
+ * set (built by an earlier muon_step with these shapes and ns_steps), so
+ * that the next such muon_step meets an invalid tile.  Synchronises the
+ * device.  Returns MUON_OK, or MUON_ERR_INVALID_ARG if no such plan, chain
+ * or tile exists.  The plan stays corrupted until muon_release().
  */
-MUON_API int muon_debug_set_tile_row(const int64_t* shapes, int n, int index, int i0);
+MUON_API int muon_debug_set_tile_row(const int64_t* shapes, int n, int ns_steps, int index, int i0);
 
 #ifdef __cplusplus
 }

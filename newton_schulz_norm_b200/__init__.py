@@ -33,7 +33,8 @@ EXPORTS = ("muon_step", "muon_orthogonalize", "muon_momentum_normalize", "muon_g
            "muon_profile_end", "muon_momentum_normalize_noalloc", "muon_adamw_step",
            "muon_step_mirrored", "muon_guard_check")
 
-PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "adamw")
+PROFILE_KINDS = ("momentum_norm_cast", "gram", "poly", "xupdate", "xupdate_final", "apply", "adamw",
+                 "ns_chain")
 
 _STATUS = {0: "MUON_OK", -1: "MUON_ERR_INVALID_ARG", -2: "MUON_ERR_UNSUPPORTED",
            -3: "MUON_ERR_CUDA", -4: "MUON_ERR_NOMEM", -5: "MUON_ERR_TIMEOUT"}

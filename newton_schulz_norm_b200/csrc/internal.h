@@ -88,10 +88,14 @@ struct alignas(64) NsProblem {
 };
 
 struct NsTile {
-  int prob;   // index into the NsProblem array
-  int i0;     // first output row
-  int j0;     // first output column
-  int kc;     // number of BK slices
+  int prob;       // index into the NsProblem array
+  int i0;         // first output row
+  int j0;         // first output column
+  int kc;         // number of BK slices
+  int op;         // NsOp of this tile
+  int wait_idx;   // chain launch: counter (in NsLaunch::deps) to wait for, or -1
+  int wait_need;  //   ... until it reaches this value (16 per tile of the phase before)
+  int done_idx;   // chain launch: counter to count this tile's stores in, or -1
 };
 
 struct FinalTable {
@@ -104,6 +108,10 @@ struct NsLaunch {
   const NsTile* tiles;
   int ntiles;
   int nprobs;                // entries of probs (checked builds validate tile.prob)
+  // Chain launches: one completion counter per (phase, matrix), zeroed before
+  // the launch; tiles name them by index (checked builds validate < ndeps).
+  int* deps;
+  int ndeps;
   int final_mode;
   // Final FINAL_PARAM launch only: one tensor map per matrix (indexed by
   // NsProblem::slot) over the stored fp32 parameters, 32 x 32 boxes with
@@ -216,8 +224,8 @@ struct AdamWLaunch {
 };
 
 // ---------------------------------------------------------------- launchers
-cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
-                           cudaStream_t stream);
+cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cudaStream_t stream,
+                           bool cooperative = false);
 cudaError_t ns_gemm_setup(int device);
 int ns_gemm_max_pairs();
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);

@@ -151,7 +151,7 @@ struct K1Plan {
   K1Info* info = nullptr;
   K1Item* items = nullptr;
   int nitems = 0;
-  int* counters = nullptr;  // [1 + 2n]: head, done[n], ready[n]
+  int* counters = nullptr;  // [1 + 2n]: head, done[n], ready[n]; then the chain's deps
   double* partials = nullptr;
   double* norms = nullptr;
   int n = 0;
@@ -168,6 +168,13 @@ struct Plan {
   NsPhase gram[2], poly, upd[2];
   K1Plan k1;
   std::vector<size_t> guards;                // guard band offsets in mem
+  // Chain tile lists (device), one per number of iterations used so far.
+  struct Chain {
+    std::unique_ptr<DevBlock> mem;
+    int ntiles = 0;
+  };
+  std::map<int, Chain> chains;
+  int* deps = nullptr;                       // 3 kMaxSteps n chain counters
   // Parameter tensor maps of the last X update, one device block per set of
   // parameter pointers, most recently used first (at most kParamMapSets).
   struct ParamMaps {
@@ -196,7 +203,8 @@ std::map<int, std::unique_ptr<DeviceCtx>> g_ctx;
 
 // ---------------------------------------------------------------- profiling events
 enum ProfKind : int {
-  PK_K1 = 0, PK_GRAM = 1, PK_POLY = 2, PK_UPDATE = 3, PK_FINAL = 4, PK_APPLY = 5, PK_ADAMW = 6
+  PK_K1 = 0, PK_GRAM = 1, PK_POLY = 2, PK_UPDATE = 3, PK_FINAL = 4, PK_APPLY = 5, PK_ADAMW = 6,
+  PK_CHAIN = 7
 };
 
 struct ProfRecord {
@@ -282,15 +290,57 @@ unsigned long long limit_ns() {
 
 // Gram / poly tiles (TILE_M x BN, one per CTA pair): only tiles holding some
 // entry on or above the diagonal.
-void sym_tiles(std::vector<NsTile>& t, int prob, long long m, int kc) {
+void sym_tiles(std::vector<NsTile>& t, int prob, long long m, int kc, int op) {
   for (long long i0 = 0; i0 < m; i0 += TILE_M)
     for (long long j0 = 0; j0 < m; j0 += BN)
-      if (std::min(j0 + BN - 1, m - 1) >= i0) t.push_back({prob, (int)i0, (int)j0, kc});
+      if (std::min(j0 + BN - 1, m - 1) >= i0) t.push_back({prob, (int)i0, (int)j0, kc, op, -1, 0, -1});
 }
 
 void full_tiles(std::vector<NsTile>& t, int prob, long long m, long long n, int kc) {
   for (long long i0 = 0; i0 < m; i0 += TILE_M)
-    for (long long j0 = 0; j0 < n; j0 += BN) t.push_back({prob, (int)i0, (int)j0, kc});
+    for (long long j0 = 0; j0 < n; j0 += BN)
+      t.push_back({prob, (int)i0, (int)j0, kc, OP_UPDATE, -1, 0, -1});
+}
+
+// The chain launch of ns_steps iterations: every Gram, polynomial and update
+// tile except the last update's, phase after phase (phase q = 3 k + {0 Gram,
+// 1 polynomial, 2 update} of iteration k), each phase listing the matrices
+// in one order, costliest first, so that the static round-robin share of
+// the pairs ends evenly and each matrix's phases come in sequence.  A tile
+// of phase q > 0 of matrix i waits for counter (q-1) n + i to reach 16 x the
+// tiles of phase q-1 of matrix i (the 8 epilogue warps of both CTAs of a
+// pair count each tile once each); every tile counts itself in q n + i.
+// Problem indices address the plan's five problem arrays laid end to end:
+// Gram from X[0] at 0, Gram from X[1] at n, update from X[0] at 2n, update
+// from X[1] at 3n, polynomial at 4n.
+std::vector<NsTile> chain_tiles(const std::vector<Geom>& geom, int ns_steps) {
+  const int n = (int)geom.size();
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  auto cost = [&](int i) { return (double)geom[i].m * geom[i].m * (3.0 * geom[i].n + geom[i].m); };
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost(a) > cost(b); });
+  std::vector<NsTile> out, one;
+  std::vector<int> prev_count(n, 0), count(n, 0);
+  const int nphases = 3 * ns_steps - 1;
+  for (int q = 0; q < nphases; ++q) {
+    const int kind = q % 3, par = (q / 3) & 1;
+    for (int i : order) {
+      const Geom& g = geom[i];
+      one.clear();
+      if (kind == 0) sym_tiles(one, par * n + i, g.m, (int)cdiv(g.n, BK), OP_GRAM);
+      else if (kind == 1) sym_tiles(one, 4 * n + i, g.m, (int)cdiv(g.m, BK), OP_POLY);
+      else full_tiles(one, (2 + par) * n + i, g.m, g.n, (int)cdiv(g.m, BK));
+      for (NsTile& t : one) {
+        t.wait_idx = q > 0 ? (q - 1) * n + i : -1;
+        t.wait_need = q > 0 ? 2 * EPI_WARPS * prev_count[i] : 0;
+        t.done_idx = q * n + i;
+      }
+      count[i] = (int)one.size();
+      out.insert(out.end(), one.begin(), one.end());
+    }
+    prev_count = count;
+  }
+  return out;
 }
 
 // K1 work queue.  Pass-2 items of a matrix wait until its norm is known,
@@ -347,11 +397,11 @@ struct TileLists {
 TileLists plan_tiles(const std::vector<Geom>& geom) {
   TileLists t;
   const int n = (int)geom.size();
-  for (int i = 0; i < n; ++i) sym_tiles(t.gram, i, geom[i].m, (int)cdiv(geom[i].n, BK));
+  for (int i = 0; i < n; ++i) sym_tiles(t.gram, i, geom[i].m, (int)cdiv(geom[i].n, BK), OP_GRAM);
   // Longest reduction first so the static round-robin ends evenly.
   std::stable_sort(t.gram.begin(), t.gram.end(),
                    [](const NsTile& x, const NsTile& y) { return x.kc > y.kc; });
-  for (int i = 0; i < n; ++i) sym_tiles(t.poly, i, geom[i].m, (int)cdiv(geom[i].m, BK));
+  for (int i = 0; i < n; ++i) sym_tiles(t.poly, i, geom[i].m, (int)cdiv(geom[i].m, BK), OP_POLY);
   for (int i = 0; i < n; ++i) full_tiles(t.upd, i, geom[i].m, geom[i].n, (int)cdiv(geom[i].m, BK));
   return t;
 }
@@ -387,7 +437,8 @@ Layout plan_layout(const std::vector<Geom>& geom, bool with_ns, const TileLists*
   }
   L.k1info = a.take(sizeof(K1Info) * n);
   L.k1items = a.take(sizeof(K1Item) * 2 * L.k1tiles);
-  L.counters = a.take(sizeof(int) * (1 + 2 * n));
+  // K1 counters, then one chain counter per (phase, matrix)
+  L.counters = a.take(sizeof(int) * (1 + 2 * n + 3 * (size_t)kMaxSteps * n));
   L.partials = a.take(sizeof(double) * L.k1tiles);
   L.norms = a.take(sizeof(double) * n);
   L.total = a.off;
@@ -548,6 +599,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, long long k1_slack,
   P->k1.partials = reinterpret_cast<double*>(base + lay.partials);
   P->k1.norms = reinterpret_cast<double*>(base + lay.norms);
   P->k1.npartials = (int)lay.k1tiles;
+  P->deps = P->k1.counters + 1 + 2 * n;
   if (cudaMemcpy(P->k1.info, info.data(), sizeof(K1Info) * n, cudaMemcpyHostToDevice) != cudaSuccess)
     return MUON_ERR_CUDA;
   if (cudaMemcpy(P->k1.items, items.data(), sizeof(K1Item) * items.size(), cudaMemcpyHostToDevice) !=
@@ -605,10 +657,13 @@ int k1_grid(DeviceCtx* ctx, int nitems) {
   return std::max(1, std::min(nitems, ctx->num_sms * ctx->k1_blocks_per_sm));
 }
 
+// zero_deps: how many chain counters after the K1 counters to zero as well
+// (the same memset), for the chain launch that follows.
 int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, int nesterov,
-           cudaStream_t stream) {
+           cudaStream_t stream, int zero_deps = 0) {
   const int n = P->k1.n;
-  if (cudaMemsetAsync(P->k1.counters, 0, sizeof(int) * (1 + 2 * n), stream) != cudaSuccess)
+  if (cudaMemsetAsync(P->k1.counters, 0, sizeof(int) * (1 + 2 * n + (size_t)zero_deps), stream) !=
+      cudaSuccess)
     return MUON_ERR_CUDA;
   static thread_local K1Launch L;   // large (12 KB); kept off the stack
   L.info = P->k1.info;
@@ -631,56 +686,86 @@ int run_k1(DeviceCtx* ctx, Plan* P, const K1Ptrs* ptrs, int mode, float beta, in
   return cuda_err(launch_k1(L, k1_grid(ctx, L.nitems), stream));
 }
 
-// The Newton-Schulz chain; the last update writes `final_mode` through F
-// (through the parameter tensor maps `pmaps` when given).
+// The chain tile list of ns_steps iterations for this plan (built and
+// uploaded on first use; blocking copies, so before any capture).
+int get_chain(Plan* P, int ns_steps, const Plan::Chain** out) {
+  auto it = P->chains.find(ns_steps);
+  if (it == P->chains.end()) {
+    std::vector<NsTile> tiles = chain_tiles(P->geom, ns_steps);
+    Plan::Chain c;
+    c.ntiles = (int)tiles.size();
+    c.mem.reset(new DevBlock());
+    const size_t bytes = sizeof(NsTile) * std::max<size_t>(1, tiles.size());
+    if (cudaMalloc(&c.mem->ptr, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_NOMEM;
+    }
+    c.mem->bytes = bytes;
+    if (!tiles.empty() &&
+        cudaMemcpy(c.mem->ptr, tiles.data(), sizeof(NsTile) * tiles.size(), cudaMemcpyHostToDevice) !=
+            cudaSuccess)
+      return MUON_ERR_CUDA;
+    it = P->chains.emplace(ns_steps, std::move(c)).first;
+  }
+  *out = &it->second;
+  return MUON_OK;
+}
+
+// Chain counters run_k1 must zero before the chain launch of ns_steps.
+int chain_deps(const Plan* P, int ns_steps) {
+  return ns_steps > 0 ? (3 * ns_steps - 1) * (int)P->geom.size() : 0;
+}
+
+// The Newton-Schulz iterations: one chain launch for every phase but the
+// last update, then the last update, which writes `final_mode` through F
+// (through the parameter tensor maps `pmaps` when given).  The chain's
+// counters were zeroed by run_k1 (zero_deps = chain_deps).
 int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mode,
            const FinalTable* F, cudaStream_t stream, const CUtensorMap* pmaps = nullptr,
            float* const* mirrors = nullptr, int n_mirrors = 0) {
+  const int n = (int)P->geom.size();
+  const Plan::Chain* chain = nullptr;
+  int rc = get_chain(P, ns_steps, &chain);
+  if (rc) return rc;
   NsLaunch L;
-  L.nprobs = (int)P->geom.size();
+  L.probs = P->gram[0].probs;            // the five problem arrays, end to end
+  L.nprobs = 5 * n;
+  L.deps = P->deps;
+  L.ndeps = 3 * kMaxSteps * n;
   L.pmaps = nullptr;
   L.mirrors = nullptr;
   L.n_mirrors = 0;
-  L.mirror_stride = (int)P->geom.size();
+  L.mirror_stride = n;
   L.ca = co[0];
   L.cb = co[1];
   L.cc = co[2];
   L.limit_ns = limit_ns();
   L.status = ctx->status;
-  for (int s = 0; s < ns_steps; ++s) {
-    const int par = s & 1;
-    L.final_mode = FINAL_NONE;
-    L.probs = P->gram[par].probs;
-    L.tiles = P->gram[par].tiles;
-    L.ntiles = P->gram[par].ntiles;
-    cudaError_t e;
-    {
-      ProfScope ps(PK_GRAM, stream);
-      e = launch_ns_gemm(OP_GRAM, L, nullptr, pair_grid(ctx, L.ntiles), stream);
-    }
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
-    L.probs = P->poly.probs;
-    L.tiles = P->poly.tiles;
-    L.ntiles = P->poly.ntiles;
-    {
-      ProfScope ps(PK_POLY, stream);
-      e = launch_ns_gemm(OP_POLY, L, nullptr, pair_grid(ctx, L.ntiles), stream);
-    }
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
-    L.probs = P->upd[par].probs;
-    L.tiles = P->upd[par].tiles;
-    L.ntiles = P->upd[par].ntiles;
-    L.final_mode = (s == ns_steps - 1) ? final_mode : FINAL_NONE;
-    L.pmaps = (s == ns_steps - 1) ? pmaps : nullptr;
-    L.mirrors = (s == ns_steps - 1) ? mirrors : nullptr;
-    L.n_mirrors = (s == ns_steps - 1) ? n_mirrors : 0;
-    {
-      ProfScope ps(L.final_mode == FINAL_NONE ? PK_UPDATE : PK_FINAL, stream);
-      e = launch_ns_gemm(OP_UPDATE, L, F, pair_grid(ctx, L.ntiles), stream);
-    }
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
+  L.final_mode = FINAL_NONE;
+  L.tiles = reinterpret_cast<const NsTile*>(chain->mem->ptr);
+  L.ntiles = chain->ntiles;
+  cudaError_t e;
+  {
+    ProfScope ps(PK_CHAIN, stream);
+    e = launch_ns_gemm(L, nullptr, pair_grid(ctx, L.ntiles), stream, /*cooperative=*/true);
   }
-  return MUON_OK;
+  if (e != cudaSuccess) return MUON_ERR_CUDA;
+  const NsPhase& last = P->upd[(ns_steps - 1) & 1];
+  L.probs = last.probs;
+  L.nprobs = n;
+  L.deps = nullptr;
+  L.ndeps = 0;
+  L.tiles = last.tiles;
+  L.ntiles = last.ntiles;
+  L.final_mode = final_mode;
+  L.pmaps = pmaps;
+  L.mirrors = mirrors;
+  L.n_mirrors = n_mirrors;
+  {
+    ProfScope ps(PK_FINAL, stream);
+    e = launch_ns_gemm(L, F, pair_grid(ctx, L.ntiles), stream);
+  }
+  return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
 int run_apply(Plan* P, int mode, void* const* dst, const float* scale, cudaStream_t stream) {
@@ -809,7 +894,7 @@ int step_group(DeviceCtx* ctx, float* const* params, const float* const* grads, 
     const double s = std::sqrt(std::max(1.0, (double)geom[i].r / (double)geom[i].c));
     F.scale[i] = (float)((double)lr * s);
   }
-  rc = run_k1(ctx, P, ptrs.data(), K1_MOMENTUM, beta, nesterov, stream);
+  rc = run_k1(ctx, P, ptrs.data(), K1_MOMENTUM, beta, nesterov, stream, chain_deps(P, ns_steps));
   if (rc) return rc;
   if (ns_steps == 0) {
     std::vector<void*> dst(params, params + n);
@@ -996,7 +1081,7 @@ int muon_orthogonalize(const float* x, void* out, int out_is_bf16, int64_t rows,
   p.buf = nullptr;
   p.x0 = P->X[0];
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rc = run_k1(ctx, P, &p, K1_PLAIN, 0.f, 0, s);
+  rc = run_k1(ctx, P, &p, K1_PLAIN, 0.f, 0, s, chain_deps(P, ns_steps));
   if (rc) return rc;
   const int mode = out_is_bf16 ? FINAL_OUT_BF16 : FINAL_OUT_F32;
   if (ns_steps == 0) {
@@ -1072,7 +1157,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
     if (op == OP_UPDATE)
       full_tiles(tiles, 0, M, N, kc);
     else
-      sym_tiles(tiles, 0, M, kc);
+      sym_tiles(tiles, 0, M, kc, op);
     const size_t bytes = 256 + sizeof(NsProblem) + sizeof(NsTile) * tiles.size();
     if (cudaMalloc(&np->mem.ptr, bytes) != cudaSuccess) {
       cudaGetLastError();
@@ -1099,6 +1184,8 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
   }
   NsLaunch L;
   L.nprobs = 1;
+  L.deps = nullptr;
+  L.ndeps = 0;
   L.pmaps = nullptr;
   L.mirrors = nullptr;
   L.n_mirrors = 0;
@@ -1112,7 +1199,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
   L.cc = cc;
   L.limit_ns = limit_ns();
   L.status = ctx->status;
-  return cuda_err(launch_ns_gemm(op, L, nullptr, pair_grid(ctx, L.ntiles),
+  return cuda_err(launch_ns_gemm(L, nullptr, pair_grid(ctx, L.ntiles),
                                  static_cast<cudaStream_t>(stream)));
 }
 
@@ -1260,7 +1347,7 @@ const char* muon_version(void) {
 }
 
 #ifdef MUON_BOUNDS_CHECK
-int muon_debug_set_tile_row(const int64_t* shapes, int n, int index, int i0) {
+int muon_debug_set_tile_row(const int64_t* shapes, int n, int ns_steps, int index, int i0) {
   if (check_shapes(shapes, n) || n < 1 || n > MUON_MAX_GROUP) return MUON_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceCtx* ctx = nullptr;
@@ -1268,14 +1355,16 @@ int muon_debug_set_tile_row(const int64_t* shapes, int n, int index, int i0) {
   if (rc) return rc;
   auto it = ctx->plans.find(shape_key('S', make_geom(shapes, n)));
   if (it == ctx->plans.end()) return MUON_ERR_INVALID_ARG;
-  NsPhase& ph = it->second->poly;
-  if (index < 0 || index >= ph.ntiles) return MUON_ERR_INVALID_ARG;
+  auto ch = it->second->chains.find(ns_steps);
+  if (ch == it->second->chains.end()) return MUON_ERR_INVALID_ARG;
+  if (index < 0 || index >= ch->second.ntiles) return MUON_ERR_INVALID_ARG;
+  NsTile* tiles = reinterpret_cast<NsTile*>(ch->second.mem->ptr);
   if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
   NsTile t;
-  if (cudaMemcpy(&t, ph.tiles + index, sizeof(t), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(&t, tiles + index, sizeof(t), cudaMemcpyDeviceToHost) != cudaSuccess)
     return MUON_ERR_CUDA;
   t.i0 = i0;
-  if (cudaMemcpy(ph.tiles + index, &t, sizeof(t), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpy(tiles + index, &t, sizeof(t), cudaMemcpyHostToDevice) != cudaSuccess)
     return MUON_ERR_CUDA;
   return MUON_OK;
 }

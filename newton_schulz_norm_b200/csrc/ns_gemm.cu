@@ -30,7 +30,18 @@
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
 // overlap the main loop of the next.  The last update moves the fp32
 // parameter blocks through a per-warp ring of TMA loads and stores instead.
-// Every wait is bounded.
+//
+// Every tile carries its operation, so one launch can run several phases:
+// the chain launch runs every Gram, polynomial and X-update tile of all
+// iterations but the last update, in phase order.  A tile of phase q of
+// matrix i waits (producer: before its first operand load; epilogue: before
+// reading its input) until every tile of phase q-1 of matrix i has been
+// stored, which the epilogue warps count in a per-(phase, matrix) counter
+// after their stores complete (release / acquire at GPU scope, with a proxy
+// fence on both sides since the stores and loads are TMA's).  Within one
+// launch a matrix's phases thus follow one another, while other matrices'
+// tiles fill the GPU, instead of a launch boundary and a full drain between
+// phases.  Every wait is bounded.
 #include <cstdio>
 
 #include "internal.h"
@@ -79,17 +90,44 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
 
 // This lane's row of the epilogue input: 32 bf16 at (row, col0 .. col0+31)
 // as four 16-byte loads (zeros outside the matrix).
+// The chain launch reads inputs that other CTAs of the same launch wrote, so
+// it may not use the non-coherent (read-only) path: its loads are plain
+// weak ld.global, which the GPU-scope acquire that precedes them orders after
+// the writers' release (L1 lines included).  Such loads still allocate in
+// L1, which matters: each lane reads 64 contiguous bytes in four 16-byte
+// loads, and L2-only loads cost every X update about 85 us on GPT-2 124M.
+__device__ __forceinline__ uint4 ld_global_weak(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned short ld_global_weak_u16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.u16 %0, [%1];" : "=h"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <bool COHERENT = false>
 __device__ __forceinline__ void load_row(const __nv_bfloat16* src, long long ld, int row, int col0,
                                          int M, int N, uint4 (&r)[4]) {
   const __nv_bfloat16* p = src + (long long)row * ld + col0;
   if (row < M && col0 + 32 <= N) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) r[q] = __ldg(reinterpret_cast<const uint4*>(p) + q);
+    for (int q = 0; q < 4; ++q)
+      r[q] = COHERENT ? ld_global_weak(reinterpret_cast<const uint4*>(p) + q)
+                      : __ldg(reinterpret_cast<const uint4*>(p) + q);
     return;
   }
   uint16_t h[32];
 #pragma unroll
-  for (int e = 0; e < 32; ++e) h[e] = (row < M && col0 + e < N) ? __bfloat16_as_ushort(p[e]) : 0;
+  for (int e = 0; e < 32; ++e)
+    h[e] = (row < M && col0 + e < N)
+               ? (COHERENT ? ld_global_weak_u16(p + e) : __bfloat16_as_ushort(p[e]))
+               : 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     r[q].x = h[8 * q + 0] | ((uint32_t)h[8 * q + 1] << 16);
@@ -322,7 +360,19 @@ __device__ __forceinline__ void mirror_block(const NsLaunch& L, const NsProblem&
   }
 }
 
-template <int OP, bool FINAL, bool MIRROR = false>
+// Waits, bounded by limit_ns, until the counter reaches `need`; acquire at
+// GPU scope.
+__device__ __forceinline__ bool wait_count(const int* p, int need, uint64_t limit_ns) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= need) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+template <bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
   constexpr int NST = FINAL ? FINAL_STAGES : STAGES;            // main-loop ring depth
   constexpr int EPI_REGION = FINAL ? FINAL_EPI_BYTES : EPI_STAGE_BYTES;   // per epilogue warp
@@ -385,7 +435,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     int bad = 0;
     for (int t = pair + (int)threadIdx.x * npairs; t < L.ntiles; t += (int)blockDim.x * npairs) {
       const NsTile tl = L.tiles[t];
-      bool ok = tl.prob >= 0 && tl.prob < L.nprobs;
+      bool ok = tl.prob >= 0 && tl.prob < L.nprobs && tl.op >= OP_GRAM && tl.op <= OP_UPDATE &&
+                (FINAL ? tl.op == OP_UPDATE : true) && tl.wait_idx < L.ndeps && tl.done_idx < L.ndeps;
       if (ok) {
         const NsProblem& Q = L.probs[tl.prob];
         ok = tl.i0 >= 0 && tl.i0 < Q.M && tl.j0 >= 0 && tl.j0 < Q.N && tl.kc > 0 &&
@@ -410,6 +461,15 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
         const NsProblem* P = L.probs + tile.prob;
+        if (tile.wait_idx >= 0) {
+          // The operands were written by the previous phase in this launch.
+          if (!wait_count(L.deps + tile.wait_idx, tile.wait_need, limit)) {
+            record_status(L.status, MUON_ERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          fence_proxy_async();                     // ... and TMA must see them
+        }
         const int arow = tile.i0 + (int)rank * BM;           // this CTA's rows of A
         const int bcol = tile.j0 + (int)rank * (BN / 2);     // this CTA's half of B
         for (int kc = 0; kc < tile.kc; ++kc) {
@@ -432,7 +492,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 #pragma unroll
           for (int q = 0; q < BM / BOX; ++q)
             tma_load_2d_pair(sA + q * BOX_BYTES, &P->tmA, fb, k0, arow + q * BOX);
-          if (OP == OP_UPDATE) {
+          if (tile.op == OP_UPDATE) {
             // B operand = X[k0:k0+64, bcol:bcol+128], MN-major: boxes along columns.
 #pragma unroll
             for (int q = 0; q < (BN / 2) / BOX; ++q)
@@ -470,9 +530,10 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t idesc = (OP == OP_UPDATE) ? kIdescMN : kIdescK;
       for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
+        const bool mn = tile.op == OP_UPDATE;
+        const uint32_t idesc = mn ? kIdescMN : kIdescK;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit)) {
           record_status(L.status, MUON_ERR_TIMEOUT);
           break;
@@ -494,7 +555,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             // 16 elements moves the start 32 bytes inside the swizzle atom.
             const uint64_t adesc = smem_desc_sw128(sA + kk * 32, 16, 1024);
             uint64_t bdesc;
-            if (OP == OP_UPDATE) {
+            if (mn) {
               // MN-major B: 64-column blocks one box (8 KB) apart, 8-row K
               // groups 1 KB apart; a K step of 16 rows moves 2 KB.
               bdesc = smem_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
@@ -672,18 +733,26 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     for (int t = pair; t < L.ntiles; t += npairs) {
       const NsTile tile = L.tiles[t];
       const NsProblem& P = L.probs[tile.prob];
+      const int op = FINAL ? OP_UPDATE : tile.op;
       const int M = P.M, N = P.N;
       const int rbase = tile.i0 + (int)rank * BM + quarter * 32;
       const int row = rbase + lane;
       const int cbase = tile.j0 + half * (CHUNKS_PER_WARP * 32);
-      // Epilogue input (this lane's row), fetched before the accumulator is ready.
-      constexpr int NPRE = (OP == OP_GRAM) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
-      uint4 ein[NPRE > 0 ? NPRE : 1][4];
+      // Epilogue input (this lane's row), fetched before the accumulator is
+      // ready; in a chain launch only once the phase that wrote it is done.
+      // The lanes wait independently (lane 0 may still be counting the last
+      // tile) and agree on failure in one vote before any warp-wide step.
+      bool fail = !FINAL && op != OP_GRAM && tile.wait_idx >= 0 &&
+                  !wait_count(L.deps + tile.wait_idx, tile.wait_need, limit);
+      const int npre = fail ? 0 : (op == OP_GRAM) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
+      uint4 ein[FINAL ? 1 : CHUNKS_PER_WARP][4];
 #pragma unroll
-      for (int cc = 0; cc < NPRE; ++cc) load_row(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
+      for (int cc = 0; cc < (FINAL ? 1 : CHUNKS_PER_WARP); ++cc)
+        if (cc < npre) load_row<!FINAL>(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
       float pcur[32];
       if (FINAL) final_load(P, F, L.final_mode, rbase, cbase, lane, pcur);
-      if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
+      if (!fail) fail = !mbar_wait(tfull_bar(acc), acc_phase, limit);
+      if (__any_sync(0xffffffffu, fail)) {
         record_status(L.status, MUON_ERR_TIMEOUT);
         break;
       }
@@ -725,7 +794,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 #pragma unroll
       for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
         const int col0 = cbase + cc * 32;
-        uint4 (&ecur)[4] = ein[NPRE > 0 ? cc : 0];
+        uint4 (&ecur)[4] = ein[FINAL ? 0 : cc];
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + cc * 32, v);
         tmem_ld_wait();
@@ -733,11 +802,11 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         float x[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(v[c]);
-        if (OP != OP_GRAM) {
+        if (op != OP_GRAM) {
           float in[32];
 #pragma unroll
           for (int q = 0; q < 4; ++q) unpack8(ecur[q], in + 8 * q);
-          if (OP == OP_POLY) {
+          if (op == OP_POLY) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) x[c] = fmaf(L.cc, x[c], L.cb * in[c]);
           } else {
@@ -745,7 +814,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             for (int c = 0; c < 32; ++c) x[c] = fmaf(L.ca, in[c], x[c]);
           }
         }
-        if (OP == OP_GRAM || OP == OP_POLY) {
+        if (op == OP_GRAM || op == OP_POLY) {
           // Symmetric output.  rbase and col0 are multiples of 32, so this
           // block lies above the diagonal (stored and mirrored), on it
           // (symmetrised, stored once) or below it (owned by another tile).
@@ -786,6 +855,15 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         acc = 0;
         acc_phase ^= 1u;
       }
+      if (!FINAL && tile.done_idx >= 0 && lane == 0) {
+        // Once this warp's stores of the tile have landed, count them for
+        // the next phase (each of the pair's 16 epilogue warps once per
+        // tile).  Only lane 0 waits; the other lanes go on to the next
+        // tile's input and accumulator, where lane 0 catches up.
+        bulk_wait_group_all();
+        fence_proxy_async();
+        red_release_gpu_add(L.deps + tile.done_idx, 1);
+      }
     }
     }
     // Stores must finish reading shared memory (and land) before the CTA exits.
@@ -805,34 +883,29 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
   }
 }
 
-template <int OP>
+// Gram, polynomial and X-update tiles, each tile naming its operation: one
+// phase per launch (stage entry points) or the whole chain of phases.
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
-  ns_gemm_body<OP, false>(L, nullptr);
+  ns_gemm_body<false>(L, nullptr);
 }
 
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     ns_gemm_final_kernel(const __grid_constant__ NsLaunch L, const __grid_constant__ FinalTable F) {
-  ns_gemm_body<OP_UPDATE, true>(L, &F);
+  ns_gemm_body<true>(L, &F);
 }
 
 // The last update that also writes every parameter block to its mirrors.
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     ns_gemm_final_mirror_kernel(const __grid_constant__ NsLaunch L,
                                 const __grid_constant__ FinalTable F) {
-  ns_gemm_body<OP_UPDATE, true, true>(L, &F);
+  ns_gemm_body<true, true>(L, &F);
 }
 
 }  // namespace
 
 cudaError_t ns_gemm_setup(int /*device*/) {
   cudaError_t e;
-  e = cudaFuncSetAttribute(ns_gemm_kernel<OP_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ns_gemm_kernel<OP_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ns_gemm_kernel<OP_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)GEMM_SMEM_BYTES);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -856,33 +929,35 @@ int ns_gemm_max_pairs() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel<OP_UPDATE>, &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     return 0;
   }
   return n;
 }
 
-// Launched as clusters of two CTAs (the MMA pair); grid is even.
-cudaError_t launch_ns_gemm(int op, const NsLaunch& L, const FinalTable* F, int grid,
-                           cudaStream_t stream) {
+// Launched as clusters of two CTAs (the MMA pair); grid is even.  A launch
+// whose tiles wait on one another (the chain) is cooperative, so that every
+// CTA it waits on is resident at the same time.
+cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cudaStream_t stream,
+                           bool cooperative) {
   if (L.ntiles <= 0) return cudaSuccess;
+  const bool fin = L.final_mode != FINAL_NONE;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = (op == OP_UPDATE && L.final_mode != FINAL_NONE) ? FINAL_SMEM_BYTES
-                                                                         : GEMM_SMEM_BYTES;
+  cfg.dynamicSmemBytes = fin ? FINAL_SMEM_BYTES : GEMM_SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (op == OP_GRAM) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_GRAM>, L);
-  if (op == OP_POLY) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_POLY>, L);
-  if (L.final_mode == FINAL_NONE) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OP_UPDATE>, L);
+  cfg.numAttrs = cooperative ? 2 : 1;
+  if (!fin) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel, L);
   if (L.n_mirrors > 0) {
     // Mirrors are written only from the shared-memory parameter ring.
     if (L.final_mode != FINAL_PARAM || L.pmaps == nullptr) return cudaErrorInvalidValue;

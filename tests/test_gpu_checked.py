@@ -38,7 +38,7 @@ def libs():
     chk.muon_guard_check.restype = ctypes.c_int64
     chk.muon_guard_check.argtypes = []
     chk.muon_debug_set_tile_row.restype = i
-    chk.muon_debug_set_tile_row.argtypes = [I64P, i, i, i]
+    chk.muon_debug_set_tile_row.argtypes = [I64P, i, i, i, i]
     chk.muon_version.restype = ctypes.c_char_p
     yield m, chk
     chk.muon_release()
@@ -86,15 +86,15 @@ def test_checked_build_turns_a_planted_tile_into_an_error(libs):
     assert chk.muon_status(None) == 0
     flat = [v for s in wl.shapes for v in s]
     sh = (ctypes.c_int64 * len(flat))(*flat)
-    # tile 0 of the polynomial phase: rows from 1024 on, past the 768 rows of its matrix
-    assert chk.muon_debug_set_tile_row(sh, len(wl.shapes), 0, 1024) == 0
+    # tile 0 of the chain (a Gram tile of a 768-row matrix): rows from 1024 on
+    assert chk.muon_debug_set_tile_row(sh, len(wl.shapes), wl.ns_steps, 0, 1024) == 0
     assert _step(chk, P, G, B, wl.shapes, wl) == 0
     torch.cuda.synchronize()
     assert chk.muon_status(None) == -1                      # MUON_ERR_INVALID_ARG
     assert chk.muon_guard_check() == 0
     assert bool(torch.isfinite(torch.cat([b.flatten() for b in B])).all())
     chk.muon_release()                                     # drop the corrupted plan
-    assert chk.muon_debug_set_tile_row(sh, len(wl.shapes), 0, 0) == -1   # no plan any more
+    assert chk.muon_debug_set_tile_row(sh, len(wl.shapes), wl.ns_steps, 0, 0) == -1   # no plan
 
 
 def test_guards_hold_after_the_largest_plans(libs):

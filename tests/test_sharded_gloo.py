@@ -1,10 +1,10 @@
 """Matrix-sharded Muon (newton_schulz_norm_b200.sharded) on CPU: the partition,
 and the all-gather path with two and three gloo ranks.
 
-The per-rank optimizer step is a stand-in here (the CUDA step needs a GPU);
-what is tested is the host logic around it: every matrix is stepped by
-exactly one rank, only owners keep momentum, and after the all-gather every
-rank holds every updated matrix.
+The CUDA step needs a GPU, so each rank steps its matrices with the oracle
+(the same per-matrix arithmetic, on the CPU): after the all-gather every rank
+must hold exactly what the oracle gives for every matrix stepped in one
+process, only owners keep momentum, and every matrix is stepped once.
 """
 import os
 import socket
@@ -51,10 +51,23 @@ def test_partition_single_rank_and_errors():
 
 
 def _fake_step(params, grads, bufs, lr, beta, nesterov, ns_steps, **kw):
-    # stand-in for the CUDA step: momentum and a plain update, in place
+    # a plain momentum update, in place (layout tests only)
     for p, g, b in zip(params, grads, bufs):
         b.mul_(beta).add_(g)
         p.sub_(lr * b)
+
+
+def _oracle_step(params, grads, bufs, lr, beta, nesterov, ns_steps, coeffs=None, **kw):
+    """The Muon step of the oracle on CPU tensors, in place: what each rank's
+    CUDA step computes for its own matrices."""
+    from oracle import muon_step_ref
+    extra = {} if coeffs is None else {"coeffs": coeffs}
+    p_new, b_new = muon_step_ref([p.numpy() for p in params], [g.numpy() for g in grads],
+                                 [b.numpy() for b in bufs], lr=lr, beta=beta, nesterov=nesterov,
+                                 ns_steps=ns_steps, **extra)
+    for p, b, pn, bn in zip(params, bufs, p_new, b_new):
+        p.copy_(torch.from_numpy(pn))
+        b.copy_(torch.from_numpy(bn))
 
 
 def _worker(rank, world, port, out):
@@ -64,23 +77,27 @@ def _worker(rank, world, port, out):
     import torch.distributed as dist
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    shapes = [(6, 10), (10, 6), (7, 7), (3, 20), (20, 3), (1, 5), (9, 4)]
-    sm = ShardedMuon(shapes, device="cpu", step_fn=_fake_step)
+    from oracle import muon_step_ref
+    shapes = [(6, 10), (10, 6), (7, 7), (3, 20), (20, 3), (1, 5), (9, 4), (24, 40)]
+    sm = ShardedMuon(shapes, device="cpu", step_fn=_oracle_step)
     rng = np.random.default_rng(0)                          # same values on every rank
-    p0 = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    p0 = [(rng.standard_normal(s) * 0.02).astype(np.float32) for s in shapes]
     for v, a in zip(sm.params, p0):
         v.copy_(torch.from_numpy(a))
     grads = [[torch.from_numpy(rng.standard_normal(s).astype(np.float32)) for s in shapes]
              for _ in range(2)]
     for g in grads:
-        sm.step(g, lr=0.1, beta=0.5)
-    # expected, computed here for every matrix: two momentum steps
+        sm.step(g, lr=0.02, beta=0.95)
+    # expected: the oracle over every matrix in one process, two steps
+    want_p = p0
+    want_b = [np.zeros(s, np.float32) for s in shapes]
+    for g in grads:
+        want_p, want_b = muon_step_ref(want_p, [t.numpy() for t in g], want_b, lr=0.02, beta=0.95)
     ok = True
-    for i, s in enumerate(shapes):
-        b1 = grads[0][i].numpy()
-        b2 = 0.5 * b1 + grads[1][i].numpy()
-        want = p0[i] - 0.1 * b1 - 0.1 * b2
-        ok &= np.allclose(sm.params[i].numpy(), want, rtol=0, atol=1e-6)
+    for i in range(len(shapes)):
+        ok &= np.array_equal(sm.params[i].numpy(), want_p[i])
+        if i in sm.bufs:
+            ok &= np.array_equal(sm.bufs[i].numpy(), want_b[i])
     ok &= sorted(sm.bufs) == sm.owned                         # momentum only where owned
     ok &= all(sm.owner[i] == rank for i in sm.owned)
     # every rank ends with the same flat buffer
@@ -102,7 +119,7 @@ def test_gloo_ranks_step_own_matrices_and_gather(world):
                        start_method="spawn")
     v = out.numpy()
     assert all(v[2 * r] == 1.0 for r in range(world)), v
-    assert sum(v[2 * r + 1] for r in range(world)) == 7      # every matrix owned once
+    assert sum(v[2 * r + 1] for r in range(world)) == 8      # every matrix owned once
 
 
 def test_single_process_layout_without_group():
