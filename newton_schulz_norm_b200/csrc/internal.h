@@ -55,6 +55,7 @@ constexpr size_t GEMM_SMEM_BYTES =
 // parameter blocks moved by TMA (32 x 32 fp32, 128-byte swizzle).
 constexpr int FINAL_STAGES = 3;
 constexpr int P_RING = 4;                    // parameter blocks per epilogue warp
+constexpr int P_AHEAD = P_RING - 2;          // chunks whose blocks are loaded ahead
 constexpr int P_BLOCK_BYTES = 32 * 32 * 4;
 constexpr int FINAL_EPI_BYTES = P_RING * P_BLOCK_BYTES;   // per epilogue warp
 constexpr size_t FINAL_SMEM_BYTES =
@@ -224,8 +225,9 @@ struct AdamWLaunch {
 };
 
 // ---------------------------------------------------------------- launchers
+// op: the NsOp of every tile of the launch, or -1 for a chain launch.
 cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cudaStream_t stream,
-                           bool cooperative = false);
+                           int op);
 cudaError_t ns_gemm_setup(int device);
 int ns_gemm_max_pairs();
 cudaError_t launch_k1(const K1Launch& L, int grid, cudaStream_t stream);

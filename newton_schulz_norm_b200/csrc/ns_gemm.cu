@@ -91,7 +91,8 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
 // This lane's row of the epilogue input: 32 bf16 at (row, col0 .. col0+31)
 // as four 16-byte loads (zeros outside the matrix).
 // The chain launch reads inputs that other CTAs of the same launch wrote, so
-// it may not use the non-coherent (read-only) path: its loads are plain
+// it may not use the non-coherent (read-only) path that one-phase launches
+// use for inputs of an earlier launch: its loads are plain
 // weak ld.global, which the GPU-scope acquire that precedes them orders after
 // the writers' release (L1 lines included).  Such loads still allocate in
 // L1, which matters: each lane reads 64 contiguous bytes in four 16-byte
@@ -372,7 +373,22 @@ __device__ __forceinline__ bool wait_count(const int* p, int need, uint64_t limi
   }
 }
 
-template <bool FINAL, bool MIRROR = false>
+// OPS names the operations the launch's tiles may have: one (a per-phase
+// launch, or the final update: the operation is then a compile-time constant
+// and the kernel carries only that epilogue) or all three (the chain launch,
+// which reads each tile's operation).
+constexpr int OPS_GRAM = 1 << OP_GRAM, OPS_POLY = 1 << OP_POLY, OPS_UPDATE = 1 << OP_UPDATE;
+constexpr int OPS_ALL = OPS_GRAM | OPS_POLY | OPS_UPDATE;
+
+template <int OPS>
+__device__ __forceinline__ int tile_op(const NsTile& t) {
+  if constexpr (OPS == OPS_GRAM) return OP_GRAM;
+  else if constexpr (OPS == OPS_POLY) return OP_POLY;
+  else if constexpr (OPS == OPS_UPDATE) return OP_UPDATE;
+  else return t.op;
+}
+
+template <int OPS, bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
   constexpr int NST = FINAL ? FINAL_STAGES : STAGES;            // main-loop ring depth
   constexpr int EPI_REGION = FINAL ? FINAL_EPI_BYTES : EPI_STAGE_BYTES;   // per epilogue warp
@@ -492,7 +508,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 #pragma unroll
           for (int q = 0; q < BM / BOX; ++q)
             tma_load_2d_pair(sA + q * BOX_BYTES, &P->tmA, fb, k0, arow + q * BOX);
-          if (tile.op == OP_UPDATE) {
+          if (tile_op<OPS>(tile) == OP_UPDATE) {
             // B operand = X[k0:k0+64, bcol:bcol+128], MN-major: boxes along columns.
 #pragma unroll
             for (int q = 0; q < (BN / 2) / BOX; ++q)
@@ -532,7 +548,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       bool ok = true;
       for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
-        const bool mn = tile.op == OP_UPDATE;
+        const bool mn = tile_op<OPS>(tile) == OP_UPDATE;
         const uint32_t idesc = mn ? kIdescMN : kIdescK;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit)) {
           record_status(L.status, MUON_ERR_TIMEOUT);
@@ -592,9 +608,10 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     if (FINAL && L.pmaps != nullptr && L.final_mode == FINAL_PARAM) {
       // ---- last iteration, parameter blocks through a per-warp TMA ring.
       // Chunk h of this warp (4 per tile, tiles in the CTA's round-robin
-      // order) owns ring slot h % P_RING.  The block for chunk h + 2 is loaded
-      // while chunk h is combined; a slot is reloaded only after the store
-      // that last used it has finished reading shared memory.
+      // order) owns ring slot h % P_RING.  The block for chunk h + P_AHEAD is
+      // loaded while chunk h is combined; that slot last held chunk
+      // h + P_AHEAD - P_RING = h - 2, whose store has finished reading shared
+      // memory once at most one store group (chunk h - 1's) is still reading.
       uint8_t* ring = stg8;
       const uint32_t ring_s = smem_addr(ring);
       const uint32_t pbar0 = pbar_base + 8u * (ew * P_RING);
@@ -625,8 +642,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         }
         pending |= 1u << b;
       };
-      issue(0);
-      issue(1);
+      for (int h = 0; h < P_AHEAD; ++h) issue(h);
       int acc = 0;
       uint32_t acc_phase = 0;
       uint4 ecur[4], enext[4];
@@ -647,7 +663,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         }
         if (lane == 0) bulk_wait_group_read<1>();   // the store of chunk h - 2 has read its slot
         __syncwarp();
-        issue(h + 2);
+        issue(h + P_AHEAD);
         if (cc + 1 < CHUNKS_PER_WARP) load_row(P.epi, P.ld_epi, row, col0 + 32, P.M, P.N, enext);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
@@ -733,7 +749,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     for (int t = pair; t < L.ntiles; t += npairs) {
       const NsTile tile = L.tiles[t];
       const NsProblem& P = L.probs[tile.prob];
-      const int op = FINAL ? OP_UPDATE : tile.op;
+      const int op = tile_op<OPS>(tile);
       const int M = P.M, N = P.N;
       const int rbase = tile.i0 + (int)rank * BM + quarter * 32;
       const int row = rbase + lane;
@@ -748,7 +764,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       uint4 ein[FINAL ? 1 : CHUNKS_PER_WARP][4];
 #pragma unroll
       for (int cc = 0; cc < (FINAL ? 1 : CHUNKS_PER_WARP); ++cc)
-        if (cc < npre) load_row<!FINAL>(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
+        if (cc < npre) load_row<OPS == OPS_ALL>(P.epi, P.ld_epi, row, cbase + cc * 32, M, N, ein[cc]);
       float pcur[32];
       if (FINAL) final_load(P, F, L.final_mode, rbase, cbase, lane, pcur);
       if (!fail) fail = !mbar_wait(tfull_bar(acc), acc_phase, limit);
@@ -883,31 +899,34 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
   }
 }
 
-// Gram, polynomial and X-update tiles, each tile naming its operation: one
-// phase per launch (stage entry points) or the whole chain of phases.
+// Gram, polynomial or X-update tiles: one phase per launch (OPS one
+// operation), or the whole chain of phases (OPS_ALL).
+template <int OPS>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ NsLaunch L) {
-  ns_gemm_body<false>(L, nullptr);
+  ns_gemm_body<OPS, false>(L, nullptr);
 }
 
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     ns_gemm_final_kernel(const __grid_constant__ NsLaunch L, const __grid_constant__ FinalTable F) {
-  ns_gemm_body<true>(L, &F);
+  ns_gemm_body<OPS_UPDATE, true>(L, &F);
 }
 
 // The last update that also writes every parameter block to its mirrors.
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     ns_gemm_final_mirror_kernel(const __grid_constant__ NsLaunch L,
                                 const __grid_constant__ FinalTable F) {
-  ns_gemm_body<true, true>(L, &F);
+  ns_gemm_body<OPS_UPDATE, true, true>(L, &F);
 }
 
 }  // namespace
 
 cudaError_t ns_gemm_setup(int /*device*/) {
   cudaError_t e;
-  e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  for (auto k : {ns_gemm_kernel<OPS_GRAM>, ns_gemm_kernel<OPS_POLY>, ns_gemm_kernel<OPS_UPDATE>,
+                 ns_gemm_kernel<OPS_ALL>}) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMM_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+  }
   e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)FINAL_SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -929,18 +948,20 @@ int ns_gemm_max_pairs() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel, &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, ns_gemm_kernel<OPS_ALL>, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     return 0;
   }
   return n;
 }
 
-// Launched as clusters of two CTAs (the MMA pair); grid is even.  A launch
-// whose tiles wait on one another (the chain) is cooperative, so that every
-// CTA it waits on is resident at the same time.
+// Launched as clusters of two CTAs (the MMA pair); grid is even.  `op` is
+// the one operation of every tile, or -1 for a chain launch (tiles of all
+// three, waiting on one another), which is cooperative so that every CTA a
+// wait depends on is resident at the same time.
 cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cudaStream_t stream,
-                           bool cooperative) {
+                           int op) {
+  const bool cooperative = op < 0;
   if (L.ntiles <= 0) return cudaSuccess;
   const bool fin = L.final_mode != FINAL_NONE;
   cudaLaunchConfig_t cfg = {};
@@ -957,7 +978,12 @@ cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cud
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 2 : 1;
-  if (!fin) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel, L);
+  if (!fin) {
+    if (op == OP_GRAM) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OPS_GRAM>, L);
+    if (op == OP_POLY) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OPS_POLY>, L);
+    if (op == OP_UPDATE) return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OPS_UPDATE>, L);
+    return cudaLaunchKernelEx(&cfg, ns_gemm_kernel<OPS_ALL>, L);
+  }
   if (L.n_mirrors > 0) {
     // Mirrors are written only from the shared-memory parameter ring.
     if (L.final_mode != FINAL_PARAM || L.pmaps == nullptr) return cudaErrorInvalidValue;
