@@ -56,6 +56,7 @@ constexpr size_t GEMM_SMEM_BYTES =
 constexpr int FINAL_STAGES = 3;
 constexpr int P_RING = 4;                    // parameter blocks per epilogue warp
 constexpr int P_AHEAD = P_RING - 2;          // chunks whose blocks are loaded ahead
+constexpr int E_AHEAD = 1;                   // chunks whose a*X input is loaded ahead
 constexpr int P_BLOCK_BYTES = 32 * 32 * 4;
 constexpr int FINAL_EPI_BYTES = P_RING * P_BLOCK_BYTES;   // per epilogue warp
 constexpr size_t FINAL_SMEM_BYTES =

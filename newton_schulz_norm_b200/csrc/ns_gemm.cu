@@ -643,9 +643,21 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         pending |= 1u << b;
       };
       for (int h = 0; h < P_AHEAD; ++h) issue(h);
+      // The epilogue input (a X) of chunk h + E_AHEAD is loaded while chunk
+      // h is combined, across tile boundaries, from a ring of registers:
+      // eb[0] is the current chunk's.
+      uint4 eb[E_AHEAD + 1][4];
+      auto in_load = [&](int h, uint4 (&dst)[4]) {
+        if (h >= nch) return;
+        const NsProblem* Pp;
+        int rb, c0;
+        chunk_info(h, Pp, rb, c0);
+        load_row(Pp->epi, Pp->ld_epi, rb + lane, c0, Pp->M, Pp->N, dst);
+      };
+#pragma unroll
+      for (int k = 0; k < E_AHEAD; ++k) in_load(k, eb[k]);
       int acc = 0;
       uint32_t acc_phase = 0;
-      uint4 ecur[4], enext[4];
       for (int h = 0; h < nch; ++h) {
         const int cc = h % CHUNKS_PER_WARP;
         const NsProblem* Pp;
@@ -654,7 +666,6 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         const NsProblem& P = *Pp;
         const int row = rb + lane;
         if (cc == 0) {
-          load_row(P.epi, P.ld_epi, row, col0, P.M, P.N, ecur);
           if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
             record_status(L.status, MUON_ERR_TIMEOUT);
             break;
@@ -664,7 +675,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         if (lane == 0) bulk_wait_group_read<1>();   // the store of chunk h - 2 has read its slot
         __syncwarp();
         issue(h + P_AHEAD);
-        if (cc + 1 < CHUNKS_PER_WARP) load_row(P.epi, P.ld_epi, row, col0 + 32, P.M, P.N, enext);
+        in_load(h + E_AHEAD, eb[E_AHEAD]);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
                                half * (CHUNKS_PER_WARP * 32) + cc * 32, v);
@@ -681,7 +692,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           } else {
             float in[32], xb[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) unpack8(ecur[q], in + 8 * q);
+            for (int q = 0; q < 4; ++q) unpack8(eb[0][q], in + 8 * q);
 #pragma unroll
             for (int c = 0; c < 32; ++c)
               xb[c] = __bfloat162float(__float2bfloat16_rn(fmaf(L.ca, in[c], __uint_as_float(v[c]))));
@@ -726,10 +737,11 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         }
         if (lane == 0) bulk_commit_group();        // one group per chunk, empty or not
         if (stop) break;
-        if (cc + 1 < CHUNKS_PER_WARP) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) ecur[q] = enext[q];
-        } else {
+        for (int k = 0; k < E_AHEAD; ++k)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) eb[k][q] = eb[k + 1][q];
+        if (cc + 1 == CHUNKS_PER_WARP) {
           tc_fence_before_sync();
           mbar_arrive_remote(map_to_cta(tempty_bar(acc), 0));
           if (++acc == 2) {
