@@ -311,14 +311,44 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_oracle_block(wl, params, grads, bufs, idx):
-    """Time the oracle on the given matrices (one step); returns seconds."""
+def cpu_oracle_block(wl, params, grads, bufs, idx, keep=None):
+    """Time the oracle on the given matrices (one step); returns seconds.
+    With ``keep`` (a dict), also stores the oracle's new parameters and
+    buffers there, for the parity spot check."""
     from oracle import muon_step_ref
     t0 = time.perf_counter()
-    muon_step_ref([params[i] for i in idx], [grads[i] for i in idx], [bufs[i] for i in idx],
-                  lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps,
-                  coeffs=wl.coeffs)
-    return time.perf_counter() - t0
+    p_new, b_new = muon_step_ref([params[i] for i in idx], [grads[i] for i in idx],
+                                 [bufs[i] for i in idx], lr=wl.lr, beta=wl.beta,
+                                 nesterov=wl.nesterov, ns_steps=wl.ns_steps, coeffs=wl.coeffs)
+    secs = time.perf_counter() - t0
+    if keep is not None:
+        keep.update(idx=list(idx), p=p_new, b=b_new)
+    return secs
+
+
+def parity_spot_check(torch, muon, wl, params, grads, bufs, ref, dev):
+    """The GPU step on the oracle's sample (same inputs, fresh copies): the
+    relative Frobenius error of each matrix's update and the largest relative
+    error of the momentum buffers, reported beside the timing."""
+    idx = ref["idx"]
+    P = [torch.from_numpy(params[i]).to(dev) for i in idx]
+    G = [torch.from_numpy(grads[i]).to(dev) for i in idx]
+    B = [torch.from_numpy(bufs[i]).to(dev) for i in idx]
+    muon.step(P, G, B, lr=wl.lr, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps,
+              coeffs=wl.coeffs)
+    torch.cuda.synchronize()
+    upd, buf = [], []
+    for k, i in enumerate(idx):
+        p0 = params[i].astype(np.float64)
+        dg = P[k].cpu().numpy().astype(np.float64) - p0
+        dr = ref["p"][k].astype(np.float64) - p0
+        upd.append(float(np.linalg.norm(dg - dr) / max(np.linalg.norm(dr), 1e-300)))
+        br = ref["b"][k].astype(np.float64)
+        buf.append(float(np.max(np.abs(B[k].cpu().numpy() - br)) / max(np.max(np.abs(br)), 1e-300)))
+    return {"matrices": idx, "update_rel_fro": upd, "buf_rel_max": max(buf),
+            "bars": {"update": 1e-2 if wl.buf_std == 0 else 2e-2, "buf": 1e-6},
+            "how": "one step of the GPU on the CPU baseline's sample (first gradient set), "
+                   "against the oracle's result"}
 
 
 def parallelism(world: int) -> str:
@@ -559,9 +589,10 @@ def run_ours(args, wl, rank, world):
 
     # CPU oracle baseline on a bounded sample (rank 0, N = 1 only), before GPU work
     cpu_base = None
+    oracle_out = {}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         idx = list(range(min(4, wl.n_matrices)))
-        secs = cpu_oracle_block(wl, params, grad_sets[0], bufs, idx)
+        secs = cpu_oracle_block(wl, params, grad_sets[0], bufs, idx, keep=oracle_out)
         cpu_base = {"value": 1e3 * secs * wl.n_matrices / len(idx), "unit": "ms",
                     "cores": blas_threads(), "kind": "oracle",
                     "sample": f"oracle on matrices {idx}, 1 step, {secs:.1f} s, "
@@ -718,6 +749,8 @@ def run_ours(args, wl, rank, world):
     peaks = load_peaks()
     adamw = None if args.no_adamw else measure_adamw(args, rank, dev, stream, barrier,
                                                       max_over_ranks, peaks)
+    parity = (parity_spot_check(torch, muon, wl, params, grad_sets[0], bufs, oracle_out, dev)
+              if oracle_out else None)
 
     # ---- roofline of the dominant kernel
     work = per_launch_work(wl)
@@ -777,6 +810,7 @@ def run_ours(args, wl, rank, world):
         "gpu_launches": launches,
         "clocks": clk,
         "adamw": adamw,
+        "parity": parity,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -18,7 +18,9 @@
  *     B  = bf16(b*A + c*A*A)
  *     X  = bf16(a*X + B*X)
  *   X   <- X^T if r > c
- *   p   <- p - (lr*sqrt(max(1, r/c))) * X     one fp32 rounding per element
+ *   p   <- p + fp32(-(lr*sqrt(max(1, r/c))) * X)   the increment rounded to
+ *                                             fp32, then added (a second
+ *                                             fp32 rounding)
  *
  * Default coefficients (a, b, c) = (3.4445, -4.7750, 2.0315).
  *

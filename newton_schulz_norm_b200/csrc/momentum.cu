@@ -348,7 +348,7 @@ __global__ void apply_kernel(const __grid_constant__ ApplyLaunch L) {
     const float x = __bfloat162float(x0[xo]);
     if (L.mode == FINAL_PARAM) {
       float* p = reinterpret_cast<float*>(L.dst[mat]) + e;
-      *p = fmaf(-L.scale[mat], x, *p);
+      *p = __fadd_rn(*p, __fmul_rn(-L.scale[mat], x));   // p + fp32(-s x), as the GEMM paths
     } else if (L.mode == FINAL_OUT_F32) {
       reinterpret_cast<float*>(L.dst[mat])[e] = x;
     } else {

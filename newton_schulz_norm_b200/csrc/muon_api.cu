@@ -18,6 +18,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 #ifdef MUON_BOUNDS_CHECK
 #include "muon_debug.h"
@@ -231,17 +233,27 @@ struct Profiler {
 Profiler g_prof;
 
 // Records an event pair around one launch when profiling is on.
+// Names of the launch kinds, for NVTX ranges (a profiler's timeline shows
+// each launch of this library under its name; without a profiler attached
+// an NVTX range costs a few nanoseconds of host time).
+const char* const kProfNames[] = {"muon: momentum/norm/cast", "muon: Gram",
+                                  "muon: polynomial",         "muon: X update",
+                                  "muon: final X update",     "muon: update (no NS)",
+                                  "muon: AdamW",              "muon: NS chain"};
+
 struct ProfScope {
   int kind;
   cudaStream_t stream;
   cudaEvent_t start = nullptr;
   ProfScope(int k, cudaStream_t s) : kind(k), stream(s) {
+    nvtxRangePushA(kProfNames[k]);
     if (g_prof.on) {
       start = g_prof.get();
       if (start) cudaEventRecord(start, stream);
     }
   }
   ~ProfScope() {
+    nvtxRangePop();
     if (!start) return;
     cudaEvent_t stop = g_prof.get();
     if (!stop) return;

@@ -271,7 +271,8 @@ __device__ __forceinline__ void final_apply(const NsProblem& P, const FinalTable
       float* base = reinterpret_cast<float*>(F->ptr[slot]);
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        if (rok && col0 + c < N) base[(long long)(col0 + c) * ldf + row] = fmaf(neg_scale, xb[c], pv[c]);
+        if (rok && col0 + c < N)
+          base[(long long)(col0 + c) * ldf + row] = __fadd_rn(pv[c], __fmul_rn(neg_scale, xb[c]));
     } else if (mode == FINAL_OUT_F32) {
       float* base = reinterpret_cast<float*>(F->ptr[slot]);
 #pragma unroll
@@ -303,10 +304,10 @@ __device__ __forceinline__ void final_apply(const NsProblem& P, const FinalTable
                          bf16_bits_to_float(w.y & 0xFFFFu), bf16_bits_to_float(w.y >> 16)};
     float4 o;
     if (mode == FINAL_PARAM) {
-      o.x = fmaf(neg_scale, x4[0], pv[4 * k + 0]);
-      o.y = fmaf(neg_scale, x4[1], pv[4 * k + 1]);
-      o.z = fmaf(neg_scale, x4[2], pv[4 * k + 2]);
-      o.w = fmaf(neg_scale, x4[3], pv[4 * k + 3]);
+      o.x = __fadd_rn(pv[4 * k + 0], __fmul_rn(neg_scale, x4[0]));
+      o.y = __fadd_rn(pv[4 * k + 1], __fmul_rn(neg_scale, x4[1]));
+      o.z = __fadd_rn(pv[4 * k + 2], __fmul_rn(neg_scale, x4[2]));
+      o.w = __fadd_rn(pv[4 * k + 3], __fmul_rn(neg_scale, x4[3]));
     } else {
       o = make_float4(x4[0], x4[1], x4[2], x4[3]);
     }
@@ -606,12 +607,19 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     uint16_t* stg = reinterpret_cast<uint16_t*>(stg8);
     const uint32_t stg_s = smem_addr(stg8);
     if (FINAL && L.pmaps != nullptr && L.final_mode == FINAL_PARAM) {
-      // ---- last iteration, parameter blocks through a per-warp TMA ring.
-      // Chunk h of this warp (4 per tile, tiles in the CTA's round-robin
-      // order) owns ring slot h % P_RING.  The block for chunk h + P_AHEAD is
-      // loaded while chunk h is combined; that slot last held chunk
-      // h + P_AHEAD - P_RING = h - 2, whose store has finished reading shared
-      // memory once at most one store group (chunk h - 1's) is still reading.
+      // ---- last iteration, the parameter update through the TMA.
+      // Without mirrors the epilogue never reads the parameters: it writes
+      // the increment d = fp32(-lr s X) of each 32 x 32 block into a
+      // shared-memory block and a TMA reduce-add makes the memory system add
+      // it to p (p <- fp32(p + d)).  Chunk h uses block h % 2, last used by
+      // chunk h - 2, whose reduce has finished reading it once at most one
+      // bulk group (chunk h - 1's) still reads.
+      // With mirrors the final values are needed here, so the parameter
+      // blocks come through a per-warp ring of TMA loads: chunk h owns ring
+      // slot h % P_RING; the block for chunk h + P_AHEAD is loaded while
+      // chunk h is combined; that slot last held chunk h + P_AHEAD - P_RING =
+      // h - 2, whose store has finished reading once at most one store group
+      // (chunk h - 1's) is still reading.  Both forms compute fp32(p + d).
       uint8_t* ring = stg8;
       const uint32_t ring_s = smem_addr(ring);
       const uint32_t pbar0 = pbar_base + 8u * (ew * P_RING);
@@ -627,7 +635,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         return rb < Pp->M && c0 < Pp->N;
       };
       auto issue = [&](int h) {          // every lane tracks the state; lane 0 issues
-        if (h >= nch) return;
+        if (!MIRROR || h >= nch) return;
         const NsProblem* Pp;
         int rb, c0;
         if (!chunk_info(h, Pp, rb, c0)) return;
@@ -664,7 +672,6 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         int rb, col0;
         const bool live = chunk_info(h, Pp, rb, col0);
         const NsProblem& P = *Pp;
-        const int row = rb + lane;
         if (cc == 0) {
           if (!mbar_wait(tfull_bar(acc), acc_phase, limit)) {
             record_status(L.status, MUON_ERR_TIMEOUT);
@@ -682,10 +689,13 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         tmem_ld_wait();
         bool stop = false;
         if (live) {
-          const int b = h % P_RING;
-          const bool got = mbar_wait(pbar0 + 8u * b, (pphase >> b) & 1u, limit);
-          pphase ^= 1u << b;
-          pending &= ~(1u << b);
+          const int b = MIRROR ? h % P_RING : (h & 1);
+          bool got = true;
+          if (MIRROR) {
+            got = mbar_wait(pbar0 + 8u * b, (pphase >> b) & 1u, limit);
+            pphase ^= 1u << b;
+            pending &= ~(1u << b);
+          }
           if (!got) {
             record_status(L.status, MUON_ERR_TIMEOUT);
             stop = true;
@@ -706,26 +716,37 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
               for (int c = 0; c < 32; ++c) {
                 float* q = reinterpret_cast<float*>(blk + c * 128 + ((((lane >> 2) ^ (c & 7))) << 4) +
                                                     ((lane & 3) << 2));
-                *q = fmaf(neg_scale, xb[c], *q);
+                const float d = __fmul_rn(neg_scale, xb[c]);
+                *q = MIRROR ? __fadd_rn(*q, d) : d;
               }
             } else {
 #pragma unroll
               for (int qd = 0; qd < 8; ++qd) {
                 float4* q = reinterpret_cast<float4*>(blk + lane * 128 + ((qd ^ (lane & 7)) << 4));
-                float4 pv = *q;
-                pv.x = fmaf(neg_scale, xb[4 * qd + 0], pv.x);
-                pv.y = fmaf(neg_scale, xb[4 * qd + 1], pv.y);
-                pv.z = fmaf(neg_scale, xb[4 * qd + 2], pv.z);
-                pv.w = fmaf(neg_scale, xb[4 * qd + 3], pv.w);
-                *q = pv;
+                float4 d = make_float4(__fmul_rn(neg_scale, xb[4 * qd + 0]),
+                                       __fmul_rn(neg_scale, xb[4 * qd + 1]),
+                                       __fmul_rn(neg_scale, xb[4 * qd + 2]),
+                                       __fmul_rn(neg_scale, xb[4 * qd + 3]));
+                if (MIRROR) {
+                  const float4 pv = *q;
+                  d = make_float4(__fadd_rn(pv.x, d.x), __fadd_rn(pv.y, d.y), __fadd_rn(pv.z, d.z),
+                                  __fadd_rn(pv.w, d.w));
+                }
+                *q = d;
               }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
               const CUtensorMap* pm = L.pmaps + P.slot;
-              if (P.transposed) tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, rb, col0);
-              else tma_store_2d(pm, ring_s + b * P_BLOCK_BYTES, col0, rb);
+              const uint32_t src = ring_s + b * P_BLOCK_BYTES;
+              if (MIRROR) {
+                if (P.transposed) tma_store_2d(pm, src, rb, col0);
+                else tma_store_2d(pm, src, col0, rb);
+              } else {
+                if (P.transposed) tma_reduce_add_2d(pm, src, rb, col0);
+                else tma_reduce_add_2d(pm, src, col0, rb);
+              }
             }
             if constexpr (MIRROR) {
               // The block is final in shared memory (only read from here on,
