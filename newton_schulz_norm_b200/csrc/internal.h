@@ -53,7 +53,7 @@ constexpr size_t GEMM_SMEM_BYTES =
 // The last X update is bound by the fp32 parameter read-modify-write, not by
 // the tensor cores, so it trades main-loop stages for a per-warp ring of
 // parameter blocks moved by TMA (32 x 32 fp32, 128-byte swizzle).
-constexpr int FINAL_STAGES = 3;
+constexpr int FINAL_STAGES = 3;             // the last update with mirrors (parameter ring)
 constexpr int P_RING = 4;                    // parameter blocks per epilogue warp
 constexpr int P_AHEAD = P_RING - 2;          // chunks whose blocks are loaded ahead
 constexpr int E_AHEAD = 1;                   // chunks whose a*X input is loaded ahead
@@ -61,6 +61,12 @@ constexpr int P_BLOCK_BYTES = 32 * 32 * 4;
 constexpr int FINAL_EPI_BYTES = P_RING * P_BLOCK_BYTES;   // per epilogue warp
 constexpr size_t FINAL_SMEM_BYTES =
     size_t(FINAL_STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * FINAL_EPI_BYTES + 1024 + GEMM_BAR_BYTES;
+// The last update without mirrors reads no parameters: two increment blocks
+// per epilogue warp, and the space left over goes to main-loop stages.
+constexpr int REDUCE_STAGES = 4;
+constexpr int REDUCE_EPI_BYTES = 2 * P_BLOCK_BYTES;
+constexpr size_t REDUCE_SMEM_BYTES =
+    size_t(REDUCE_STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * REDUCE_EPI_BYTES + 1024 + GEMM_BAR_BYTES;
 
 enum NsOp : int { OP_GRAM = 0, OP_POLY = 1, OP_UPDATE = 2 };
 

@@ -391,8 +391,9 @@ __device__ __forceinline__ int tile_op(const NsTile& t) {
 
 template <int OPS, bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
-  constexpr int NST = FINAL ? FINAL_STAGES : STAGES;            // main-loop ring depth
-  constexpr int EPI_REGION = FINAL ? FINAL_EPI_BYTES : EPI_STAGE_BYTES;   // per epilogue warp
+  constexpr int NST = FINAL ? (MIRROR ? FINAL_STAGES : REDUCE_STAGES) : STAGES;   // ring depth
+  constexpr int EPI_REGION = FINAL ? (MIRROR ? FINAL_EPI_BYTES : REDUCE_EPI_BYTES)
+                                   : EPI_STAGE_BYTES;                          // per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;     // 128B-swizzle atoms need 1 KB alignment
@@ -961,7 +962,7 @@ cudaError_t ns_gemm_setup(int /*device*/) {
     if (e != cudaSuccess) return e;
   }
   e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)FINAL_SMEM_BYTES);
+                           (int)REDUCE_SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(ns_gemm_final_mirror_kernel,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FINAL_SMEM_BYTES);
@@ -1000,7 +1001,8 @@ cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cud
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = fin ? FINAL_SMEM_BYTES : GEMM_SMEM_BYTES;
+  cfg.dynamicSmemBytes = !fin ? GEMM_SMEM_BYTES
+                         : (L.n_mirrors > 0 ? FINAL_SMEM_BYTES : REDUCE_SMEM_BYTES);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
