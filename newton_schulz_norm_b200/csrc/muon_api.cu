@@ -772,6 +772,7 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
     ProfScope ps(kind, stream);
     e = launch_ns_gemm(L, nullptr, pair_grid(ctx, L.ntiles), stream, op);
   };
+  bool chained = false;
   if (use_chain(ctx, P, ns_steps)) {
     const Plan::Chain* chain = nullptr;
     int rc = get_chain(P, ns_steps, &chain);
@@ -786,11 +787,22 @@ int run_ns(DeviceCtx* ctx, Plan* P, int ns_steps, const float* co, int final_mod
       ProfScope ps(PK_CHAIN, stream);
       e = launch_ns_gemm(L, nullptr, pair_grid(ctx, L.ntiles), stream, /*op=*/-1);
     }
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
     L.nprobs = n;
     L.deps = nullptr;
     L.ndeps = 0;
-  } else {
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+      // The device cannot hold every CTA pair at once right now (it is shared
+      // with another context): nothing was launched, so run the phases as
+      // separate launches instead.
+      cudaGetLastError();
+      e = cudaSuccess;
+    } else if (e != cudaSuccess) {
+      return MUON_ERR_CUDA;
+    } else {
+      chained = true;
+    }
+  }
+  if (!chained) {
     for (int s = 0; s < ns_steps; ++s) {
       const int par = s & 1;
       phase(P->gram[par], OP_GRAM, PK_GRAM);

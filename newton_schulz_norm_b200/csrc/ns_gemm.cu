@@ -391,7 +391,8 @@ __device__ __forceinline__ int tile_op(const NsTile& t) {
 
 template <int OPS, bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
-  constexpr int NST = FINAL ? (MIRROR ? FINAL_STAGES : REDUCE_STAGES) : STAGES;   // ring depth
+  constexpr int NST = FINAL ? (MIRROR ? FINAL_STAGES : REDUCE_STAGES)
+                            : (OPS == OPS_POLY ? POLY_STAGES : STAGES);   // ring depth
   constexpr int EPI_REGION = FINAL ? (MIRROR ? FINAL_EPI_BYTES : REDUCE_EPI_BYTES)
                                    : EPI_STAGE_BYTES;                          // per epilogue warp
   extern __shared__ uint8_t smem_raw[];
@@ -956,11 +957,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
 cudaError_t ns_gemm_setup(int /*device*/) {
   cudaError_t e;
-  for (auto k : {ns_gemm_kernel<OPS_GRAM>, ns_gemm_kernel<OPS_POLY>, ns_gemm_kernel<OPS_UPDATE>,
-                 ns_gemm_kernel<OPS_ALL>}) {
+  for (auto k : {ns_gemm_kernel<OPS_GRAM>, ns_gemm_kernel<OPS_UPDATE>, ns_gemm_kernel<OPS_ALL>}) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMM_SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
+  e = cudaFuncSetAttribute(ns_gemm_kernel<OPS_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)POLY_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)REDUCE_SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -1001,8 +1004,8 @@ cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cud
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = !fin ? GEMM_SMEM_BYTES
-                         : (L.n_mirrors > 0 ? FINAL_SMEM_BYTES : REDUCE_SMEM_BYTES);
+  cfg.dynamicSmemBytes = fin ? (L.n_mirrors > 0 ? FINAL_SMEM_BYTES : REDUCE_SMEM_BYTES)
+                             : (op == OP_POLY ? POLY_SMEM_BYTES : GEMM_SMEM_BYTES);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
