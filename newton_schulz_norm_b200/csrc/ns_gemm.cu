@@ -491,6 +491,10 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         }
         const int arow = tile.i0 + (int)rank * BM;           // this CTA's rows of A
         const int bcol = tile.j0 + (int)rank * (BN / 2);     // this CTA's half of B
+        // A diagonal tile of a symmetric product (Gram, polynomial): both
+        // operands are rows of one matrix and this CTA's half of B is its own
+        // rows of A, so the B slice is not loaded; the MMA reads it from A.
+        const bool same_ab = tile_op<OPS>(tile) != OP_UPDATE && tile.i0 == tile.j0;
         for (int kc = 0; kc < tile.kc; ++kc) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit)) {
             record_status(L.status, MUON_ERR_TIMEOUT);
@@ -498,7 +502,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             break;
           }
           if (leader) {
-            mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+            mbar_arrive_expect_tx(full_bar(stage), same_ab ? 2 * A_STAGE_BYTES : 2 * STAGE_BYTES);
             armed_mask |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -516,7 +520,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
 #pragma unroll
             for (int q = 0; q < (BN / 2) / BOX; ++q)
               tma_load_2d_pair(sB + q * BOX_BYTES, &P->tmB, fb, bcol + q * BOX, k0);
-          } else {
+          } else if (!same_ab) {
             // B operand = rows bcol..bcol+128 of X (or A), K-major.
 #pragma unroll
             for (int q = 0; q < (BN / 2) / BOX; ++q)
@@ -552,6 +556,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const NsTile tile = L.tiles[t];
         const bool mn = tile_op<OPS>(tile) == OP_UPDATE;
+        const bool same_ab = !mn && tile.i0 == tile.j0;   // B slice = A slice (see producer)
         const uint32_t idesc = mn ? kIdescMN : kIdescK;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit)) {
           record_status(L.status, MUON_ERR_TIMEOUT);
@@ -567,7 +572,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           }
           tc_fence_after_sync();
           const uint32_t sA = sbase + stage * STAGE_BYTES;
-          const uint32_t sB = sA + A_STAGE_BYTES;
+          const uint32_t sB = same_ab ? sA : sA + A_STAGE_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             // K-major A: 128-byte rows, 8-row groups 1 KB apart; a K step of

@@ -9,7 +9,7 @@ roundings, which the chaotic iteration amplifies.  These tests show, on the
 GPT-2 block trajectory, that at step 8 both the tensor core's truncating
 accumulation and even round-to-nearest fp32 accumulation (with or without
 split-K) land more than 1e-2 from the oracle, so the GPU parity tests hold
-momentum-trajectory steps to 1.5e-2 and check separately (on the GPU) that
+momentum-trajectory steps to 2e-2 and check separately (on the GPU) that
 the GPU tracks this model step by step.
 """
 from fractions import Fraction
@@ -106,13 +106,14 @@ def test_model_rounds_like_the_oracle_when_nothing_is_inexact():
     assert rel_fro(a, b) < 2e-3            # only the fp32 epilogue roundings differ
 
 
-def _block_step8_u(i):
+def _block_u(i, step):
+    """u of matrix i at the given step (from 1) of the GPT-2 block trajectory."""
     wl = WORKLOADS["gpt2_block"]
     st = WorkloadStream(wl, seed=0)
     _, bufs = st.init()
-    for k in range(8):
+    for k in range(step):
         grads = st.next_grads()
-        if k < 7:
+        if k < step - 1:
             for j in range(len(bufs)):
                 bufs[j] = momentum_ref(grads[j], bufs[j], wl.beta, wl.nesterov)[0].astype(np.float32)
     _, u = momentum_ref(grads[i], bufs[i], wl.beta, wl.nesterov)
@@ -126,11 +127,15 @@ def test_fp32_accumulation_misses_one_percent_at_trajectory_step_8():
     accumulators, and round-to-nearest fp32 accumulation all land more than
     1e-2 from the oracle (1.34%, 1.18% and 1.05% when written), while a
     zero-momentum step stays inside it."""
-    u = _block_step8_u(0)
+    u = _block_u(0, 8)
     ref = orthogonalize_ref(u, 5, COEFFS)
     e_trunc = rel_fro(orthogonalize_tc(u, 5, COEFFS, "trunc"), ref)
     e_split = rel_fro(orthogonalize_tc(u, 5, COEFFS, "trunc", splits=4), ref)
     e_rn = rel_fro(orthogonalize_tc(u, 5, COEFFS, "rn"), ref)
     print(f"step 8: truncating {e_trunc:.4%}, split-K x4 {e_split:.4%}, nearest {e_rn:.4%}")
     assert e_trunc > e_split > e_rn > 1e-2
-    assert e_trunc < 1.5e-2
+    assert e_trunc < 2e-2
+    u1 = _block_u(0, 1)                      # zero momentum: the first step
+    e1 = rel_fro(orthogonalize_tc(u1, 5, COEFFS, "trunc"), orthogonalize_ref(u1, 5, COEFFS))
+    print(f"step 1: truncating {e1:.4%}")
+    assert e1 < 1e-2
