@@ -182,11 +182,19 @@ def recorded_traffic(kind):
 
 # ---------------------------------------------------------------- clocks
 
+def start_clocks(torch, dev):
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    clocks.start()
+    return clocks
+
+
 class ClockSampler:
-    """SM clock, power and clock-event reasons sampled every 5 ms through NVML
-    (read only) in a background thread.  Only samples taken between
-    ``load_begin()`` and ``load_end()`` (the timed region, while the GPU runs
-    the queued steps) count; falls back to ``nvidia-smi -lms 100``."""
+    """SM clock, power and clock-event reasons read through NVML (read only)
+    while the GPU runs the timed region: ``wait(event)`` samples from the
+    calling thread until the region's last event has completed, so even a
+    region of a few milliseconds holds samples.  Falls back to
+    ``nvidia-smi -lms 100`` when NVML is unavailable."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
@@ -197,64 +205,50 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.samples = []            # (sm_mhz, max_mhz, power_w, reasons_mask)
-        self.loaded = False
-        self.thread = None
         self.proc = None
         self.nvml = None
 
     def start(self):
-        import threading
         try:
             import pynvml
             pynvml.nvmlInit()
             h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
-            self.nvml = (pynvml, h)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.nvml = (pynvml, h, get_reasons, smax)
+            return
         except Exception:
             self.nvml = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def sample(self):
         if self.nvml is None:
-            try:
-                self.proc = subprocess.Popen(
-                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                     "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
-                    stderr=subprocess.DEVNULL, text=True)
-            except OSError:
-                self.proc = None
-            time.sleep(0.3)
             return
-        self.stop_flag = False
+        nv, h, get_reasons, smax = self.nvml
+        try:
+            power = nv.nvmlDeviceGetPowerUsage(h) / 1000.0 if len(self.samples) % 4 == 0 else \
+                (self.samples[-1][2] if self.samples else 0.0)
+            self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax, power,
+                                 int(get_reasons(h))))
+        except Exception:
+            pass
 
-        def run():
-            nv, h = self.nvml
-            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
-            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            power = 0.0
-            k = 0
-            while not self.stop_flag:
-                if self.loaded:
-                    try:
-                        if k % 4 == 0:          # power is the slowest query: every 4th sample
-                            power = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax,
-                                             power, int(get_reasons(h))))
-                        k += 1
-                    except Exception:
-                        pass
-                time.sleep(0.002)
-
-        self.thread = threading.Thread(target=run, daemon=True)
-        self.thread.start()
-
-    def load_begin(self):
-        self.loaded = True
-
-    def load_end(self):
-        self.loaded = False
+    def wait(self, event):
+        """Sample until ``event`` (recorded after the timed work) completes."""
+        while not event.query():
+            self.sample()
+            time.sleep(0.0005)
 
     def stop(self):
-        if self.thread is not None:
-            self.stop_flag = True
-            self.thread.join(timeout=5)
+        if self.nvml is not None:
             try:
                 self.nvml[0].nvmlShutdown()
             except Exception:
@@ -265,7 +259,8 @@ class ClockSampler:
                     "sm_min_mhz": min(sm) if sm else None,
                     "sm_max_mhz": self.samples[0][1] if self.samples else None,
                     "power_w_max": max(x[2] for x in self.samples) if self.samples else None,
-                    "samples": len(sm), "source": "NVML every ~2 ms during the timed region",
+                    "samples": len(sm),
+                    "source": "NVML, read back to back while the timed region runs",
                     "reasons": reasons}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -481,13 +476,16 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
     muon.profile_begin()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    clocks = start_clocks(torch, dev)
     e0.record(stream)
     t0 = aw.step + args.warmup
     for k in range(args.steps):
         groups[k % N_GRAD_SETS].step(t0 + k)
     e1.record(stream)
+    clocks.wait(e1)
     torch.cuda.synchronize()
     prof = muon.profile_end()
+    clk = clocks.stop()
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     kern_ms, launches = prof["adamw"]
@@ -502,6 +500,7 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
                          "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("adamw"),
                          "bytes_per_launch": per_launch, "avg_launch_ms": kern_ms / launches,
                          "peak_source": f"{peaks['source']} (burst)"},
+            "clocks": clk,
             "l2": f"inputs larger than L2: {N_GRAD_SETS} gradient sets cycled "
                   f"({N_GRAD_SETS * aw.n_elements * 4 / 1e9:.2f} GB) + 3 state arrays "
                   f"({3 * aw.n_elements * 4 / 1e9:.2f} GB)"}
@@ -640,19 +639,16 @@ def run_ours(args, wl, rank, world):
     time.sleep(0.25)
 
     # ---- timed region (device-resident): the headline value
-    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    clocks = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
-    clocks.start()
+    clocks = start_clocks(torch, dev)
     barrier()
     torch.cuda.synchronize()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    clocks.load_begin()
     evs[0].record(stream)
     for k in range(args.steps):
         muon.step(P, G[k % N_GRAD_SETS], B, **kw)
         evs[k + 1].record(stream)
+    clocks.wait(evs[-1])
     torch.cuda.synchronize()
-    clocks.load_end()
     barrier()
     clk = clocks.stop()
     ms_local = evs[0].elapsed_time(evs[-1]) / args.steps
@@ -861,11 +857,14 @@ def run_square(args, n, rank, world):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    clocks = start_clocks(torch, dev)
     e0.record(stream)
     for _ in range(args.steps):
         muon.orthogonalize(x, out=out)
     e1.record(stream)
+    clocks.wait(e1)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     ranks.barrier()
     ms = ranks.max(e0.elapsed_time(e1) / args.steps)
     if muon.status() != 0:
@@ -909,6 +908,7 @@ def run_square(args, n, rank, world):
                      "peak_source": f"{peaks['source']} (burst)", "work_per_launch": work[dom],
                      "avg_launch_ms": dom_ms / dom_n},
         "kernels": kernels,
+        "clocks": clk,
         "cpu_baseline": cpu_base,
         "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": 4 * n * n,
                 "d2h_bytes_per_step": 2 * n * n},

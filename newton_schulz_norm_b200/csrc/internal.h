@@ -32,11 +32,7 @@ constexpr int BM = 128;                     // output rows per CTA
 constexpr int TILE_M = 256;                 // output rows per CTA pair
 constexpr int BN = 256;
 constexpr int BK = 64;                      // one 128-byte swizzle row of bf16
-constexpr int STAGES = 6;                   // Gram, X update and chain launches
-// The polynomial phase (four short tiles per CTA pair) runs best with a
-// shallower ring: measured on GPT-2 124M, 41 us with 4 stages, 43 with 5,
-// 45 with 6 (the Gram and the X update are fastest with 6).
-constexpr int POLY_STAGES = 4;
+constexpr int STAGES = 6;                   // every launch but the last update
 constexpr int BOX = 64;                     // TMA box: 64 x 64 bf16 = 8 KB
 constexpr int BOX_BYTES = BOX * BOX * 2;
 constexpr int A_STAGE_BYTES = BM * BK * 2;          // 16 KB: this CTA's rows of A
@@ -53,8 +49,6 @@ constexpr int OUT_BOX = 32;                 // TMA store box: 32 x 32 bf16, 64-b
 constexpr int GEMM_BAR_BYTES = 512;
 constexpr size_t GEMM_SMEM_BYTES =
     size_t(STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
-constexpr size_t POLY_SMEM_BYTES =
-    size_t(POLY_STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;
 
 // The last X update is bound by the fp32 parameter read-modify-write, not by
 // the tensor cores, so it trades main-loop stages for a per-warp ring of

@@ -59,6 +59,7 @@ constexpr unsigned long long kDrainLimitNs = 1000000000ull;
 
 constexpr uint32_t kIdescK = idesc_bf16_f32(TILE_M, BN, 0);   // pair MMA, B K-major
 constexpr uint32_t kIdescMN = idesc_bf16_f32(TILE_M, BN, 1);  // pair MMA, B MN-major
+constexpr int HOLD_CHUNKS = BN / BK;                       // K slices of one 256-wide block: 4
 constexpr int CHUNKS_PER_WARP = BN / 32 / 2;               // 4
 
 __device__ __forceinline__ void record_status(int* status, int code) {
@@ -171,6 +172,18 @@ __device__ __forceinline__ void symmetrize_block(uint8_t* blk, int lane) {
       *reinterpret_cast<uint16_t*>(blk + sw64(r, c >> 3) + 2 * (c & 7)) = v;
     }
   }
+}
+
+// This lane's 32 epilogue inputs from a held operand slice (see hold_range):
+// row rr of this CTA's A rows, K values k0 .. k0+31.  The slice holds two
+// TMA boxes of 64 rows x 128 bytes in the 128-byte swizzle: 16-byte unit u
+// of row r sits at unit u ^ (r & 7).
+__device__ __forceinline__ void held_row(const uint8_t* sa, int rr, int k0, uint4 (&e)[4]) {
+  const uint8_t* rowp = sa + (rr >> 6) * BOX_BYTES + (rr & 63) * 128;
+  const int sw = rr & 7;
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    e[v] = *reinterpret_cast<const uint4*>(rowp + ((((k0 >> 3) + v) ^ sw) << 4));
 }
 
 // One bf16 row per lane -> staging block (row-major).
@@ -389,12 +402,32 @@ __device__ __forceinline__ int tile_op(const NsTile& t) {
   else return t.op;
 }
 
+// Held K slices.  In the one-phase polynomial launch the epilogue input is
+// a block of this CTA's own A operand: B = b A + c A^2 needs A(I, J), which
+// is its A slice (rows I) for the K range J.  Those slices come last in the
+// tile's K order (the order starts right after them and wraps), stay in the
+// ring until the epilogue has read them, and the epilogue, not the MMA
+// commit, releases them, so the input never comes from L2.  start: the
+// slice at position 0; nheld: how many.
+template <int OPS, bool FINAL>
+__device__ __forceinline__ void hold_range(const NsTile& t, int& start, int& nheld) {
+  start = 0;
+  nheld = 0;
+  if constexpr (!FINAL && OPS == OPS_POLY) {
+    const int lo = t.j0 / BK;
+    const int hi = min(lo + HOLD_CHUNKS, t.kc);
+    nheld = max(hi - lo, 0);
+    start = hi < t.kc ? hi : 0;
+  }
+}
+
 template <int OPS, bool FINAL, bool MIRROR = false>
 __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable* F) {
   constexpr int NST = FINAL ? (MIRROR ? FINAL_STAGES : REDUCE_STAGES)
-                            : (OPS == OPS_POLY ? POLY_STAGES : STAGES);   // ring depth
+                            : STAGES;   // ring depth
   constexpr int EPI_REGION = FINAL ? (MIRROR ? FINAL_EPI_BYTES : REDUCE_EPI_BYTES)
                                    : EPI_STAGE_BYTES;                          // per epilogue warp
+  constexpr bool HOLD = !FINAL && OPS == OPS_POLY;   // see hold_range
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;     // 128B-swizzle atoms need 1 KB alignment
@@ -411,6 +444,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
   constexpr int NBARS = 2 * NST + 5 + (FINAL ? EPI_WARPS * P_RING : 0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + NST * STAGE_BYTES +
                                                     EPI_WARPS * EPI_REGION + 8 * NBARS);
+  // Per stage: epilogue warps done reading it as a held slice (four per use).
+  int* hold_cnt = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -432,6 +467,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       mbar_init(tempty_bar(a), 2 * EPI_THREADS);     // leader: both CTAs' epilogues
     }
     mbar_init(drain_bar, 1);
+    if (HOLD)
+      for (int s = 0; s < NST; ++s) hold_cnt[s] = 0;
     if (FINAL)
       for (int b = 0; b < EPI_WARPS * P_RING; ++b) mbar_init(pbar_base + 8u * b, 1);
     fence_barrier_init();
@@ -489,12 +526,15 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           }
           fence_proxy_async();                     // ... and TMA must see them
         }
+        const int op = tile_op<OPS>(tile);
         const int arow = tile.i0 + (int)rank * BM;           // this CTA's rows of A
         const int bcol = tile.j0 + (int)rank * (BN / 2);     // this CTA's half of B
         // A diagonal tile of a symmetric product (Gram, polynomial): both
         // operands are rows of one matrix and this CTA's half of B is its own
         // rows of A, so the B slice is not loaded; the MMA reads it from A.
-        const bool same_ab = tile_op<OPS>(tile) != OP_UPDATE && tile.i0 == tile.j0;
+        const bool same_ab = op != OP_UPDATE && tile.i0 == tile.j0;
+        int kstart, nheld;
+        hold_range<OPS, FINAL>(tile, kstart, nheld);
         for (int kc = 0; kc < tile.kc; ++kc) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit)) {
             record_status(L.status, MUON_ERR_TIMEOUT);
@@ -511,11 +551,12 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
           const uint32_t fb = map_to_cta(full_bar(stage), 0);   // the leader's barrier
           const uint32_t sA = sbase + stage * STAGE_BYTES;
           const uint32_t sB = sA + A_STAGE_BYTES;
-          const int k0 = kc * BK;
+          const int kslice = kstart + kc < tile.kc ? kstart + kc : kstart + kc - tile.kc;
+          const int k0 = kslice * BK;
 #pragma unroll
           for (int q = 0; q < BM / BOX; ++q)
             tma_load_2d_pair(sA + q * BOX_BYTES, &P->tmA, fb, k0, arow + q * BOX);
-          if (tile_op<OPS>(tile) == OP_UPDATE) {
+          if (op == OP_UPDATE) {
             // B operand = X[k0:k0+64, bcol:bcol+128], MN-major: boxes along columns.
 #pragma unroll
             for (int q = 0; q < (BN / 2) / BOX; ++q)
@@ -558,6 +599,8 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         const bool mn = tile_op<OPS>(tile) == OP_UPDATE;
         const bool same_ab = !mn && tile.i0 == tile.j0;   // B slice = A slice (see producer)
         const uint32_t idesc = mn ? kIdescMN : kIdescK;
+        int kstart, nheld;
+        hold_range<OPS, FINAL>(tile, kstart, nheld);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit)) {
           record_status(L.status, MUON_ERR_TIMEOUT);
           break;
@@ -588,7 +631,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             }
             umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kc | kk) != 0 ? 1u : 0u);
           }
-          umma_commit_pair(empty_bar(stage), 0x3);   // both CTAs' slices free
+          if (kc < tile.kc - nheld) umma_commit_pair(empty_bar(stage), 0x3);   // both CTAs' slices free
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
@@ -786,11 +829,16 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
     } else {
     int acc = 0;
     uint32_t acc_phase = 0;
+    int it = 0;     // ring position of the tile's first K slice (as producer and MMA count)
     for (int t = pair; t < L.ntiles; t += npairs) {
       const NsTile tile = L.tiles[t];
       const NsProblem& P = L.probs[tile.prob];
       const int op = tile_op<OPS>(tile);
       const int M = P.M, N = P.N;
+      int kstart, nheld;
+      hold_range<OPS, FINAL>(tile, kstart, nheld);
+      const int held0 = it + tile.kc - nheld;      // ring position of the first held slice
+      it += tile.kc;
       const int rbase = tile.i0 + (int)rank * BM + quarter * 32;
       const int row = rbase + lane;
       const int cbase = tile.j0 + half * (CHUNKS_PER_WARP * 32);
@@ -800,7 +848,7 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
       // tile) and agree on failure in one vote before any warp-wide step.
       bool fail = !FINAL && op != OP_GRAM && tile.wait_idx >= 0 &&
                   !wait_count(L.deps + tile.wait_idx, tile.wait_need, limit);
-      const int npre = fail ? 0 : (op == OP_GRAM) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
+      const int npre = fail ? 0 : (op == OP_GRAM || HOLD) ? 0 : (FINAL ? 1 : CHUNKS_PER_WARP);
       uint4 ein[FINAL ? 1 : CHUNKS_PER_WARP][4];
 #pragma unroll
       for (int cc = 0; cc < (FINAL ? 1 : CHUNKS_PER_WARP); ++cc)
@@ -813,6 +861,34 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
         break;
       }
       tc_fence_after_sync();
+      if (HOLD) {
+        // Every MMA of the tile has completed: the held slices are read here
+        // (this half's two) and released, the fourth reader warp of a slice
+        // arriving on its empty barrier.
+#pragma unroll
+        for (int cc = 0; cc < CHUNKS_PER_WARP; ++cc) {
+          const int ci = half * (CHUNKS_PER_WARP / 2) + (cc >> 1);
+          if (ci < nheld) {
+            held_row(gbase + ((held0 + ci) % NST) * STAGE_BYTES, quarter * 32 + lane, (cc & 1) * 32,
+                     ein[cc]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int u = 0; u < CHUNKS_PER_WARP / 2; ++u) {
+            const int ci = half * (CHUNKS_PER_WARP / 2) + u;
+            if (ci < nheld) {
+              const int s = (held0 + ci) % NST;
+              __threadfence_block();
+              if ((atomicAdd(hold_cnt + s, 1) & 3) == 3) {
+                __threadfence_block();
+                mbar_arrive(empty_bar(s));
+              }
+            }
+          }
+        }
+      }
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN +
                              half * (CHUNKS_PER_WARP * 32);
       const bool rows_live = rbase < M;
@@ -962,13 +1038,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
 cudaError_t ns_gemm_setup(int /*device*/) {
   cudaError_t e;
-  for (auto k : {ns_gemm_kernel<OPS_GRAM>, ns_gemm_kernel<OPS_UPDATE>, ns_gemm_kernel<OPS_ALL>}) {
+  for (auto k : {ns_gemm_kernel<OPS_GRAM>, ns_gemm_kernel<OPS_POLY>, ns_gemm_kernel<OPS_UPDATE>,
+                 ns_gemm_kernel<OPS_ALL>}) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMM_SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
-  e = cudaFuncSetAttribute(ns_gemm_kernel<OPS_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)POLY_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ns_gemm_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)REDUCE_SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -1010,7 +1084,7 @@ cudaError_t launch_ns_gemm(const NsLaunch& L, const FinalTable* F, int grid, cud
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(GEMM_THREADS);
   cfg.dynamicSmemBytes = fin ? (L.n_mirrors > 0 ? FINAL_SMEM_BYTES : REDUCE_SMEM_BYTES)
-                             : (op == OP_POLY ? POLY_SMEM_BYTES : GEMM_SMEM_BYTES);
+                             : GEMM_SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
