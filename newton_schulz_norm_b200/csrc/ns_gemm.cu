@@ -23,13 +23,16 @@
 //   warps 2-9  the epilogue: two warps per TMEM lane quarter, each taking
 //              four 32-column chunks of its 32 rows.  A warp reads its chunk
 //              from TMEM (tcgen05.ld, one row per thread), combines it with
-//              the epilogue input (fetched before the accumulator is ready),
-//              writes bf16 rows into a 64-byte-swizzled 32x32 staging block
+//              the epilogue input (fetched before the accumulator is ready;
+//              in the polynomial launch read from operand slices held in
+//              the ring, see hold_range), writes bf16 rows into a 64-byte-swizzled 32x32 staging block
 //              and stores it with a TMA store.  Symmetric outputs store each
 //              block above the diagonal twice (as itself and mirrored).
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
-// overlap the main loop of the next.  The last update moves the fp32
-// parameter blocks through a per-warp ring of TMA loads and stores instead.
+// overlap the main loop of the next.  The last update adds its fp32
+// parameter increments with TMA reduce-adds instead (or, when mirrors need
+// the final values, moves the parameter blocks through a per-warp ring of TMA
+// loads and stores).
 //
 // Every tile carries its operation, so one launch can run several phases:
 // the chain launch runs every Gram, polynomial and X-update tile of all
