@@ -191,10 +191,12 @@ def start_clocks(torch, dev):
 
 class ClockSampler:
     """SM clock, power and clock-event reasons read through NVML (read only)
-    while the GPU runs the timed region: ``wait(event)`` samples from the
-    calling thread until the region's last event has completed, so even a
-    region of a few milliseconds holds samples.  Falls back to
-    ``nvidia-smi -lms 100`` when NVML is unavailable."""
+    while the GPU runs the timed region: a background thread samples from
+    ``begin()`` on (the host may spend the whole region queueing launches),
+    and ``wait(event)`` goes on sampling from the calling thread until the
+    region's last event has completed, so even a region of a few
+    milliseconds holds samples.  Falls back to ``nvidia-smi -lms 100`` when
+    NVML is unavailable."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
@@ -207,6 +209,9 @@ class ClockSampler:
         self.samples = []            # (sm_mhz, max_mhz, power_w, reasons_mask)
         self.proc = None
         self.nvml = None
+        self.active = False
+        self.done = False
+        self.thread = None
 
     def start(self):
         try:
@@ -217,9 +222,20 @@ class ClockSampler:
                 getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
             smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self.nvml = (pynvml, h, get_reasons, smax)
-            return
         except Exception:
             self.nvml = None
+        if self.nvml is not None:
+            import threading
+
+            def run():
+                while not self.done:
+                    if self.active:
+                        self.sample()
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -241,13 +257,20 @@ class ClockSampler:
         except Exception:
             pass
 
+    def begin(self):
+        self.active = True
+
     def wait(self, event):
         """Sample until ``event`` (recorded after the timed work) completes."""
         while not event.query():
             self.sample()
             time.sleep(0.0005)
+        self.active = False
 
     def stop(self):
+        self.done = True
+        if self.thread is not None:
+            self.thread.join(timeout=5)
         if self.nvml is not None:
             try:
                 self.nvml[0].nvmlShutdown()
@@ -477,6 +500,7 @@ def measure_adamw(args, rank, dev, stream, barrier, max_over_ranks, peaks):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks = start_clocks(torch, dev)
+    clocks.begin()
     e0.record(stream)
     t0 = aw.step + args.warmup
     for k in range(args.steps):
@@ -643,6 +667,7 @@ def run_ours(args, wl, rank, world):
     barrier()
     torch.cuda.synchronize()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    clocks.begin()
     evs[0].record(stream)
     for k in range(args.steps):
         muon.step(P, G[k % N_GRAD_SETS], B, **kw)
@@ -858,6 +883,7 @@ def run_square(args, n, rank, world):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks = start_clocks(torch, dev)
+    clocks.begin()
     e0.record(stream)
     for _ in range(args.steps):
         muon.orthogonalize(x, out=out)
