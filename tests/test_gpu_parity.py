@@ -114,7 +114,7 @@ def test_momentum_three_steps_exact_match(muon):
 # ---------------------------------------------------------------- NS stages
 
 NS_SHAPES = [(7, 20), (64, 64), (128, 256), (200, 333), (256, 1024), (768, 768), (768, 3072),
-             (130, 300), (1, 9)]
+             (130, 300), (1, 9), (600, 1000)]
 
 
 def _trace_inputs(m, n, seed):
