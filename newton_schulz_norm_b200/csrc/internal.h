@@ -44,8 +44,10 @@ constexpr int GEMM_THREADS = 64 + EPI_THREADS;  // warp 0 TMA, warp 1 MMA, warps
 constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators of BN columns
 constexpr int EPI_LD = 40;                  // padded staging pitch (bf16) of the final kernel
 constexpr int EPI_BLOCK_BYTES = 32 * 32 * 2;       // one 32 x 32 bf16 block, 64-byte swizzled
-constexpr int EPI_STAGE_BYTES = 2 * EPI_BLOCK_BYTES;   // two blocks per epilogue warp
-constexpr int OUT_BOX = 32;                 // TMA store box: 32 x 32 bf16, 64-byte swizzle
+// Per epilogue warp: a block and its mirror (symmetric outputs), or one
+// 32 x 64 block with 128-byte swizzle (X update).
+constexpr int EPI_STAGE_BYTES = 2 * EPI_BLOCK_BYTES;
+constexpr int OUT_BOX = 32;                 // TMA store box: 32 rows x 32 (or 64) bf16
 constexpr int GEMM_BAR_BYTES = 512;
 constexpr size_t GEMM_SMEM_BYTES =
     size_t(STAGES) * STAGE_BYTES + size_t(EPI_WARPS) * EPI_STAGE_BYTES + 1024 + GEMM_BAR_BYTES;

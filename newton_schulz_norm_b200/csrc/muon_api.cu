@@ -75,17 +75,21 @@ bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols
   return r == CUDA_SUCCESS;
 }
 
-// Output map for TMA stores: 32 x 32 bf16 boxes with 64-byte swizzle (the
-// layout of the epilogue's staging blocks).
-bool make_out_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld) {
+// Output map for TMA stores, in the layout of the epilogue's staging blocks:
+// 32 x 32 bf16 boxes with 64-byte swizzle (symmetric outputs, which also
+// store each block mirrored), or 32 rows x 64 columns with 128-byte swizzle
+// (X-update outputs: two chunks per store).
+bool make_out_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
+                  bool wide = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {(cuuint32_t)OUT_BOX, (cuuint32_t)OUT_BOX};
+  cuuint32_t box[2] = {(cuuint32_t)(wide ? 2 * OUT_BOX : OUT_BOX), (cuuint32_t)OUT_BOX};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -565,7 +569,7 @@ int build_plan(const std::vector<Geom>& geom, bool with_ns, long long k1_slack,
         q.ld_epi = g.ldx;
         q.out = P->X[1 - par] + P->x_off[i];
         q.ld_out = g.ldx;
-        if (!make_out_map(&q.tmOut, q.out, g.m, g.n, g.ldx)) return MUON_ERR_CUDA;
+        if (!make_out_map(&q.tmOut, q.out, g.m, g.n, g.ldx, true)) return MUON_ERR_CUDA;
         q.M = (int)g.m;
         q.N = (int)g.n;
         q.K = (int)g.m;
@@ -1234,7 +1238,7 @@ static int run_stage(int op, const uint16_t* opA, long long ldA, const uint16_t*
     q.ld_epi = ld_epi;
     q.out = reinterpret_cast<__nv_bfloat16*>(out);
     q.ld_out = ld_out;
-    if (!make_out_map(&q.tmOut, out, M, N, ld_out)) return MUON_ERR_CUDA;
+    if (!make_out_map(&q.tmOut, out, M, N, ld_out, op == OP_UPDATE)) return MUON_ERR_CUDA;
     q.M = (int)M;
     q.N = (int)N;
     q.K = (int)K;

@@ -25,9 +25,11 @@
 //              from TMEM (tcgen05.ld, one row per thread), combines it with
 //              the epilogue input (fetched before the accumulator is ready;
 //              in the polynomial launch read from operand slices held in
-//              the ring, see hold_range), writes bf16 rows into a 64-byte-swizzled 32x32 staging block
-//              and stores it with a TMA store.  Symmetric outputs store each
-//              block above the diagonal twice (as itself and mirrored).
+//              the ring, see hold_range), writes bf16 rows into a swizzled
+//              staging block and stores it with a TMA store: 32 x 32 blocks
+//              for symmetric outputs, which store each block above the
+//              diagonal twice (as itself and mirrored); 32 x 64 blocks, two
+//              chunks per store, for the X update.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
 // overlap the main loop of the next.  The last update adds its fp32
 // parameter increments with TMA reduce-adds instead (or, when mirrors need
@@ -161,6 +163,16 @@ __device__ __forceinline__ void col_to_block(uint8_t* blk, int lane, const float
   for (int c = 0; c < 32; ++c)
     *reinterpret_cast<uint16_t*>(blk + sw64(c, q) + 2 * e) =
         __bfloat16_as_ushort(__float2bfloat16_rn(x[c]));
+}
+
+// Chunk `second` (0 or 1) of a 32 x 64 bf16 staging block in the TMA 128-byte
+// swizzle (row r: bytes [128 r, 128 r + 128), 16-byte unit u at u ^ (r & 7)):
+// the lane's row, columns 32 second .. 32 second + 31.  Bank-conflict free.
+__device__ __forceinline__ void row_to_wide(uint8_t* blk, int lane, int second, const float (&x)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(blk + lane * 128 + (((4 * second + q) ^ (lane & 7)) << 4)) =
+        pack8(x + 8 * q);
 }
 
 // Diagonal block: entries below the diagonal take the value computed above
@@ -971,15 +983,20 @@ __device__ __forceinline__ void ns_gemm_body(const NsLaunch& L, const FinalTable
             bulk_commit_group();
           }
         } else {
-          uint8_t* blk = stg8 + (cc & 1) * EPI_BLOCK_BYTES;
-          if (lane == 0) bulk_wait_group_read<1>();    // the store from this block two chunks ago
-          __syncwarp();
-          row_to_block(blk, lane, x);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&P.tmOut, stg_s + (cc & 1) * EPI_BLOCK_BYTES, col0, rbase);
-            bulk_commit_group();
+          // X update: two chunks fill one 32 x 64 block, which leaves in one
+          // TMA store (half as many stores as 32 x 32 blocks).
+          if ((cc & 1) == 0) {
+            if (lane == 0) bulk_wait_group_read<0>();  // the last block's store has read it
+            __syncwarp();
+          }
+          row_to_wide(stg8, lane, cc & 1, x);
+          if ((cc & 1) == 1 || cc + 1 == CHUNKS_PER_WARP || col0 + 32 >= N) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&P.tmOut, stg_s, col0 - (cc & 1) * 32, rbase);
+              bulk_commit_group();
+            }
           }
         }
       }
